@@ -1,0 +1,133 @@
+/*
+ * condensate_attn.h - C ABI of the Condensate attention library (B200, sm_100a).
+ *
+ * The operation ("Condensate Theorem（冷凝定理）：注意力稀疏性的拓扑本质",
+ * §2.1 Definition 1, §2.2.1-§2.2.3, §2.4 Corollary 3, §5.2.2): for every
+ * query position i of a (batch, q-head),
+ *
+ *     t_ij = q_i . k_j                      (j <= i, causal)
+ *     C_i  = {0} U [max(0, i-W_i+1), i] U Top-k_i
+ *     o_i  = softmax(t_ij / sqrt(d), j in C_i) . V
+ *
+ * Top-k_i holds the m_i = min(k, max(0, i-W_i)) best candidates of
+ * [1, i-W_i] (the causal positions outside anchor and window), ranked by
+ * t_ij descending with ties going to the lower index, so that
+ * |C_i| = min(i+1, 1+W_i+k) (§2.4 Corollary 2 as an equality).  With a
+ * per-query window array W_i (§2.4 Corollary 3, W_i = 64 + 192 RepScore_i)
+ * the scalar W is ignored.  A window at least as long as the sequence (or
+ * cache) covers every causal position.
+ *
+ * Layouts (row-major, head dimension innermost, no padding):
+ *   prefill  Q [B, Hq, n, d]; K, V [B, Hkv, n, d]; O [B, Hq, n, d]
+ *            idx [B, Hq, n, C_max] int32; idx_count [B, Hq, n] int32;
+ *            W_i [B, n] int32 (optional)
+ *   decode   q [B, Hq, d]; K, V [B, Hkv, L, d] (the cache, holding the current
+ *            token at position L-1, which is the query position);
+ *            O [B, Hq, d]; idx [B, Hq, C_max]; idx_count [B, Hq];
+ *            W_i [B] int32 (optional)
+ * q-head h reads kv-head h / (Hq/Hkv) (grouped-query attention).
+ * idx rows hold C_i in ascending order, padded with -1 up to C_max.
+ * Supported: d in {64, 128}; dtype CA_F32 or CA_BF16 for Q/K/V (all three
+ * alike); O may be CA_F32 or CA_BF16; Hq/Hkv in {1, 2, 4, 8}.
+ * Scores and the softmax are accumulated in fp32; selection uses the
+ * unscaled fp32 dot product with the tie rule above.
+ *
+ * Ownership: every pointer is a device pointer owned by the caller; the
+ * library allocates nothing and keeps no global mutable state.  `stream` is a
+ * cudaStream_t (NULL = legacy default stream).  Calls are asynchronous; the
+ * returned status covers argument checks and launch errors only.
+ *
+ * Errors: arguments are validated before anything is launched (null
+ * pointers, sizes, d, group size, 16-byte alignment, C_max >= 1+W+k for the
+ * scalar window, workspace size).  Values read on the device (a W_i below
+ * 1, a W_i whose set overflows C_max, a bounded wait that ran out)
+ * set flags in the workspace's status word; condensate_attn_status() waits
+ * for the stream and reports them.  The status word is cleared at the start
+ * of every call that uses the workspace.  Inputs must be finite.
+ */
+#ifndef CONDENSATE_ATTN_H
+#define CONDENSATE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CA_API __attribute__((visibility("default")))
+#else
+#define CA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CA_OK = 0,
+  CA_ERR_INVALID_ARG = 1, /* null pointer, bad size, C_max too small        */
+  CA_ERR_UNSUPPORTED = 2, /* d, dtype or group size outside the list above  */
+  CA_ERR_ALIGNMENT = 3,   /* a tensor pointer is not 16-byte aligned         */
+  CA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required         */
+  CA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed            */
+  CA_ERR_TIMEOUT = 6,     /* a bounded device wait gave up (status query)    */
+  CA_ERR_DEVICE_ARG = 7   /* W_i out of range or set overflowing C_max      */
+} ca_status;
+
+typedef enum { CA_F32 = 0, CA_BF16 = 1 } ca_dtype;
+
+/*
+ * Bytes of device workspace needed by one prefill (is_decode = 0; n_or_L = n)
+ * or decode (is_decode = 1; n_or_L = L) call with these sizes.  W_max is the
+ * largest window the call may use.  Pure host function; returns 0 for
+ * invalid sizes.
+ */
+CA_API size_t condensate_attn_workspace_size(int is_decode, ca_dtype dtype, int B,
+                                      int n_or_L, int Hq, int Hkv, int d,
+                                      int W_max, int k);
+
+/*
+ * Causal prefill over n positions (§2.1 Definition 1 applied to every row,
+ * §5.2.2 select-then-attend).  Two launches: a fused score + Top-k pass
+ * (tcgen05 tensor cores for bf16, FFMA for fp32) and a gather + fp32 online
+ * softmax pass.  W_i may be NULL.
+ */
+CA_API ca_status condensate_attn_prefill(const void* Q, const void* K, const void* V,
+                                  ca_dtype dtype, int B, int n, int Hq,
+                                  int Hkv, int d, int W, int k,
+                                  const int32_t* W_i, void* O,
+                                  ca_dtype o_dtype, int32_t* idx,
+                                  int32_t* idx_count, int C_max,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
+ * Decode of one query per (batch, q-head) at position L-1 against an L-long
+ * cache (§2.1 Definition 1 for the last row).  Two launches: a K-streaming
+ * score pass with a per-chunk Top-k, and a merge + gather + softmax pass.
+ * W_i may be NULL.
+ */
+CA_API ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
+                                 ca_dtype dtype, int B, int L, int Hq, int Hkv,
+                                 int d, int W, int k, const int32_t* W_i,
+                                 void* O, ca_dtype o_dtype, int32_t* idx,
+                                 int32_t* idx_count, int C_max,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
+ * Waits for `stream`, then reads and clears the device status word of
+ * `workspace`: CA_OK, CA_ERR_DEVICE_ARG or CA_ERR_TIMEOUT (CA_ERR_CUDA if
+ * the wait or copy itself failed).
+ */
+CA_API ca_status condensate_attn_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+CA_API const char* condensate_attn_status_string(ca_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+CA_API int condensate_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONDENSATE_ATTN_H */

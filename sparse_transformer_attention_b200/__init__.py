@@ -1,0 +1,11 @@
+"""Condensate ("Topological") attention for NVIDIA B200 (sm_100a).
+
+The computation lives in the CUDA library `libcondensate_attn.so` behind the
+C ABI declared in `include/condensate_attn.h`; this package is its ctypes
+binding and the build step that produces it.
+"""
+from .binding import (  # noqa: F401
+    CA_BF16, CA_F32, CA_OK, CondensateError, LIB_PATH,
+    condensate_attn_decode, condensate_attn_prefill, condensate_attn_status,
+    condensate_attn_workspace_size, load, status_string,
+)

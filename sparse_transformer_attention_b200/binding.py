@@ -1,0 +1,200 @@
+"""ctypes binding of the Condensate attention C ABI (include/condensate_attn.h).
+
+Argument marshalling only: torch provides device memory and the current
+stream, every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback: if the library or a CUDA device is missing the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcondensate_attn.so")
+
+CA_OK = 0
+CA_ERR_INVALID_ARG = 1
+CA_ERR_UNSUPPORTED = 2
+CA_ERR_ALIGNMENT = 3
+CA_ERR_WORKSPACE = 4
+CA_ERR_CUDA = 5
+CA_ERR_TIMEOUT = 6
+CA_ERR_DEVICE_ARG = 7
+
+CA_F32 = 0
+CA_BF16 = 1
+
+# (name, restype, argtypes) of every entry point the header declares.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+SIGNATURES = {
+    "condensate_attn_workspace_size":
+        (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "condensate_attn_prefill":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
+              _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_decode":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
+              _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_status": (_I, [_P, _P]),
+    "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
+    "condensate_attn_version": (_I, []),
+}
+
+_lib = None
+
+
+class CondensateError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+def load(path: Optional[str] = None):
+    """Load the C-ABI library (built in-tree by sparse_transformer_attention_b200.build)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(
+            f"Condensate attention library not found at {p}; build it with "
+            "`python -m sparse_transformer_attention_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().condensate_attn_status_string(int(code)).decode()
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return CA_F32
+    if t == torch.bfloat16:
+        return CA_BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def condensate_attn_workspace_size(is_decode: bool, dtype: torch.dtype, B: int,
+                                   n_or_L: int, Hq: int, Hkv: int, d: int,
+                                   W_max: int, k: int) -> int:
+    return int(load().condensate_attn_workspace_size(
+        int(bool(is_decode)), _dt(dtype), B, n_or_L, Hq, Hkv, d, W_max, k))
+
+
+def _check(code: int, where: str):
+    if code != CA_OK:
+        raise CondensateError(code, where)
+
+
+def _require(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def condensate_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                            W: int, k: int, W_i: Optional[torch.Tensor] = None,
+                            O: Optional[torch.Tensor] = None,
+                            o_dtype: torch.dtype = torch.float32,
+                            idx: Optional[torch.Tensor] = None,
+                            idx_count: Optional[torch.Tensor] = None,
+                            C_max: Optional[int] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            stream=None) -> Tuple[torch.Tensor, torch.Tensor,
+                                                  torch.Tensor]:
+    """Causal prefill.  Q [B,Hq,n,d], K/V [B,Hkv,n,d] (fp32 or bf16, CUDA).
+
+    Returns (O [B,Hq,n,d], idx [B,Hq,n,C_max] int32, idx_count [B,Hq,n]).
+    """
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V")):
+        _require(t, nm)
+    W_max = int(W_i.max().item()) if (W_i is not None and C_max is None) else W
+    if C_max is None:
+        C_max = 1 + W_max + k
+    dev = Q.device
+    if O is None:
+        O = torch.empty((B, Hq, n, d), dtype=o_dtype, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Hq, n, C_max), dtype=torch.int32, device=dev)
+    if idx_count is None:
+        idx_count = torch.empty((B, Hq, n), dtype=torch.int32, device=dev)
+    if workspace is None:
+        ws = condensate_attn_workspace_size(False, Q.dtype, B, n, Hq, Hkv, d,
+                                            max(1, W_max), k)
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    code = load().condensate_attn_prefill(
+        _ptr(Q), _ptr(K), _ptr(V), _dt(Q.dtype), B, n, Hq, Hkv, d, int(W),
+        int(k), _ptr(W_i), _ptr(O), _dt(O.dtype), _ptr(idx), _ptr(idx_count),
+        int(C_max), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_prefill")
+    return O, idx, idx_count
+
+
+def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                           W: int, k: int, W_i: Optional[torch.Tensor] = None,
+                           O: Optional[torch.Tensor] = None,
+                           o_dtype: torch.dtype = torch.float32,
+                           idx: Optional[torch.Tensor] = None,
+                           idx_count: Optional[torch.Tensor] = None,
+                           C_max: Optional[int] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor,
+                                                 torch.Tensor]:
+    """Decode at position L-1.  q [B,Hq,d], K/V [B,Hkv,L,d] (CUDA).
+
+    Returns (O [B,Hq,d], idx [B,Hq,C_max] int32, idx_count [B,Hq]).
+    """
+    B, Hq, d = q.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    for t, nm in ((q, "q"), (K, "K"), (V, "V")):
+        _require(t, nm)
+    W_max = int(W_i.max().item()) if (W_i is not None and C_max is None) else W
+    if C_max is None:
+        C_max = min(L, 1 + W_max + k)
+    dev = q.device
+    if O is None:
+        O = torch.empty((B, Hq, d), dtype=o_dtype, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Hq, C_max), dtype=torch.int32, device=dev)
+    if idx_count is None:
+        idx_count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    if workspace is None:
+        ws = condensate_attn_workspace_size(True, q.dtype, B, L, Hq, Hkv, d,
+                                            max(1, W_max), k)
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    code = load().condensate_attn_decode(
+        _ptr(q), _ptr(K), _ptr(V), _dt(q.dtype), B, L, Hq, Hkv, d, int(W),
+        int(k), _ptr(W_i), _ptr(O), _dt(O.dtype), _ptr(idx), _ptr(idx_count),
+        int(C_max), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_decode")
+    return O, idx, idx_count
+
+
+def condensate_attn_status(workspace: torch.Tensor, stream=None) -> int:
+    """Wait for the stream and return (and clear) the device status code."""
+    return int(load().condensate_attn_status(_ptr(workspace), _stream(stream)))

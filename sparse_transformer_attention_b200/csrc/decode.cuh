@@ -1,0 +1,36 @@
+// Decode path launch interface (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ca {
+
+// About two CTAs per SM on a 148-SM B200 for the K-streaming pass.
+constexpr int kDecodeTargetCtas = 296;
+// Upper bound on merged candidates per q-head (chunks x k), so the merge
+// fits in shared memory.
+constexpr int kDecodeMaxMerge = 8192;
+
+struct DecodeArgs {
+  const void* q;
+  const void* K;
+  const void* V;
+  int B, L, Hq, Hkv, W, k;
+  const int32_t* W_i;
+  void* O;
+  int o_bf16;
+  int32_t* idx;
+  int32_t* idx_count;
+  int C_max;
+  int chunk_len, nchunks, kpow2;
+  uint64_t* cand;     // [B, Hq, nchunks, k] chunk-best keys (workspace)
+  uint32_t* status;   // device status word (workspace)
+};
+
+int decode_chunks(int B, int L, int Hkv, int k);
+int decode_chunk_len(int L, int nchunks);
+cudaError_t decode_launch(const DecodeArgs& a, bool bf16, int d,
+                          cudaStream_t stream);
+
+}  // namespace ca

@@ -1,0 +1,101 @@
+// CTA-wide exact selection on 64-bit keys (see make_key in common.cuh).
+//
+// Radix select, most significant byte first: each pass histograms the keys
+// that still match the chosen prefix and picks the byte whose bucket holds
+// the kk-th largest key.  A list stops early once its chosen bucket holds
+// exactly the keys still needed: every key of the bucket is then selected,
+// and the bucket's lower bound (prefix followed by zero bytes) separates the
+// selected keys from the others.  Several independent lists share passes and
+// barriers.
+#pragma once
+
+#include "common.cuh"
+
+namespace ca {
+
+template <int NL>
+struct SelectState {
+  uint64_t prefix[NL];
+  uint32_t need[NL];
+  uint32_t done[NL];
+  uint32_t hist[NL * 256];
+};
+
+// For each list l < NL (keys[l*stride .. l*stride + n[l])), compute T[l] such
+// that exactly kk[l] keys are >= T[l] (keys unique, kk[l] >= 1).  A list
+// with n[l] <= kk[l] gets T[l] = 0 (keep all).  n, kk and T live in shared
+// memory; every thread of the CTA must call this; on return every thread
+// may read T.
+template <int NT, int NL>
+__device__ void cta_select_thresholds(const uint64_t* keys, int stride,
+                                      const int* n, const int* kk, uint64_t* T,
+                                      SelectState<NL>* st) {
+  static_assert(NL * 32 <= NT, "one warp per list for the bucket scan");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid < NL) {
+    st->prefix[tid] = 0;
+    st->need[tid] = (uint32_t)kk[tid];
+    st->done[tid] = n[tid] <= kk[tid];
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    bool all_done = true;
+#pragma unroll
+    for (int l = 0; l < NL; ++l) all_done = all_done && st->done[l];
+    if (all_done) break;  // uniform: every thread reads the same state
+    const uint64_t hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
+    for (int b = tid; b < NL * 256; b += NT) st->hist[b] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int l = 0; l < NL; ++l) {
+      if (st->done[l]) continue;
+      const uint64_t* kl = keys + (size_t)l * stride;
+      const uint64_t pf = st->prefix[l];
+      const int nl = n[l];
+      for (int e = tid; e < nl; e += NT) {
+        uint64_t key = kl[e];
+        if ((key & hmask) == pf)
+          atomicAdd(&st->hist[l * 256 + ((uint32_t)(key >> shift) & 255u)], 1u);
+      }
+    }
+    __syncthreads();
+    if (warp < NL && !st->done[warp]) {
+      const uint32_t* h = st->hist + warp * 256;
+      uint32_t c[8], sum = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        c[t] = h[255 - 8 * lane - t];
+        sum += c[t];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const uint32_t excl = incl - sum;
+      const uint32_t nd = st->need[warp];
+      __syncwarp();
+      if (excl < nd && nd <= incl) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (acc + c[t] >= nd) {
+            const uint32_t digit = 255u - 8u * lane - t;
+            st->prefix[warp] |= (uint64_t)digit << shift;
+            st->need[warp] = nd - acc;
+            if (c[t] == nd - acc) st->done[warp] = 1u;
+            break;
+          }
+          acc += c[t];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (tid < NL) T[tid] = (n[tid] <= kk[tid]) ? 0ull : st->prefix[tid];
+  __syncthreads();
+}
+
+}  // namespace ca

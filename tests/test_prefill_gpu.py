@@ -1,0 +1,80 @@
+"""Prefill parity on the GPU: the CUDA path through the C ABI against the CPU
+oracle (all rows for small shapes, sampled rows at full size)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from gpu_common import check_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_rows(w, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for i in [0, 1, w.W - 1, w.W, w.W + 1, w.W + w.k, w.W + w.k + 1, w.n - 1]:
+        if 0 <= i < w.n:
+            rows.add((0, 0, i))
+            rows.add((w.B - 1, w.Hq - 1, i))
+    while len(rows) < count:
+        rows.add((int(rng.integers(w.B)), int(rng.integers(w.Hq)),
+                  int(rng.integers(w.n))))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def test_tiny_prefill_f32():
+    """The tiny fp32 prefill workload, every row."""
+    w = workloads.get("tiny_prefill_f32")
+    print(check_prefill(w, workloads.generate(w)))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n,W,k", [
+    (1, 1, 0), (2, 1, 1), (64, 64, 32), (65, 64, 32), (97, 64, 32),
+    (200, 1, 16), (300, 300, 8), (333, 7, 64), (1000, 64, 32), (777, 3, 1),
+])
+def test_prefill_edges(dtype, d, n, W, k):
+    w = workloads.get("prefill_gpt2s_8k").scaled(
+        dtype=dtype, d=d, n=n, W=W, k=k, B=2, Hq=4, Hkv=2, needles=2,
+        needle_gap=W)
+    print(check_prefill(w, workloads.generate(w)))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_gqa_groups(dtype):
+    w = workloads.get("prefill_gpt2s_8k").scaled(
+        dtype=dtype, n=700, B=1, Hq=8, Hkv=1, needles=4)
+    print(check_prefill(w, workloads.generate(w)))
+
+
+def test_prefill_gpt2s_small_all_rows():
+    w = workloads.get("prefill_gpt2s_8k").scaled(n=1536, B=2, Hq=3, Hkv=3)
+    print(check_prefill(w, workloads.generate(w)))
+
+
+def test_prefill_adaptive_small_all_rows():
+    w = workloads.get("prefill_adaptive_32k").scaled(n=2048, Hq=2, Hkv=2)
+    x = workloads.generate(w)
+    print(check_prefill(w, x, W_i=x["W_i"]))
+
+
+def test_prefill_bf16_output():
+    w = workloads.get("prefill_gpt2s_8k").scaled(n=600, B=1, Hq=2, Hkv=2)
+    print(check_prefill(w, workloads.generate(w), o_dtype=torch.bfloat16,
+                        tol=1e-2 + 2.0 ** -6))
+
+
+def test_prefill_gpt2s_8k_sampled():
+    """The GPT-2-small 8K prefill workload at full size, sampled rows."""
+    w = workloads.get("prefill_gpt2s_8k")
+    x = workloads.generate(w)
+    print(check_prefill(w, x, sel=_sample_rows(w, 1500, 0)))
+
+
+def test_prefill_adaptive_32k_sampled():
+    """The adaptive-window 32K prefill workload at full size, sampled rows."""
+    w = workloads.get("prefill_adaptive_32k")
+    x = workloads.generate(w)
+    print(check_prefill(w, x, W_i=x["W_i"], sel=_sample_rows(w, 600, 1)))
