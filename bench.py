@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the Condensate attention hot path on B200.
+
+One step = one call of the library's public entry point for the workload
+(decode: score pass + per-chunk Top-k + merge + gather/softmax; prefill:
+score + Top-k pass + gather/softmax) over one batch of seeded synthetic
+input already resident in device memory.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+With N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the workload on its own GPU ("replicas only": the
+path has no exchange step); the step time is the maximum over ranks.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "decode ms @131K/1M ctx; prefill tokens/s; % of HBM / tensor roofline"
+DEFAULT_WORKLOAD = "decode_131k"
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                   choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        m = json.load(open(path))
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- work model
+def work_model(w):
+    """Algorithmic work per launch of each kernel (see the design notes)."""
+    es = 2 if w.dtype == "bf16" else 4
+    if w.kind == "decode":
+        L = w.n
+        size = min(L, 1 + w.W + w.k)
+        return {
+            "decode_score_topk": ("hbm", w.B * w.Hkv * L * w.d * es,
+                                  "K bytes scored: B*Hkv*L*d*elem"),
+            "decode_merge_attend": ("hbm", w.B * w.Hq * size * 2 * w.d * es,
+                                    "K and V rows of C_i: B*Hq*|C|*2*d*elem"),
+        }
+    n = w.n
+    flops = w.B * w.Hq * w.d * n * (n + 1)
+    return {
+        "prefill_score_topk_tc": ("tensor", flops,
+                                  "causal score FLOPs: B*H*d*n*(n+1)"),
+        "prefill_score_topk_f32": ("alu", flops,
+                                   "causal score FLOPs: B*H*d*n*(n+1)"),
+        "prefill_gather": ("hbm", w.B * w.Hq * n * (w.C_max * 4 + w.d * 4),
+                           "idx and O writes: B*H*n*(C_max*4 + d*4)"),
+    }
+
+
+def step_units(w):
+    return w.B if w.kind == "decode" else w.B * w.n  # tokens per step
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "sparse_transformer_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        t = json.load(open(path))
+    except ValueError:
+        return None
+    e = t.get(f"{kernel}/{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                   "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd.insert(1, f"--id={self.uuid}")
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import sparse_transformer_attention_b200 as ca
+    from sparse_transformer_attention_b200 import binding
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.get(args.workload)
+    x = workloads.generate(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tdt)
+    Q, K, V = to(x["Q"]), to(x["K"]), to(x["V"])
+    W_i = None if x["W_i"] is None else torch.from_numpy(x["W_i"]).to(dev)
+    W_max = w.W_max
+    decode = w.kind == "decode"
+    if decode:
+        C_max = min(w.n, 1 + W_max + w.k)
+        O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+        idx = torch.empty((w.B, w.Hq, C_max), dtype=torch.int32, device=dev)
+        cnt = torch.empty((w.B, w.Hq), dtype=torch.int32, device=dev)
+    else:
+        C_max = 1 + W_max + w.k
+        O = torch.empty((w.B, w.Hq, w.n, w.d), dtype=torch.float32, device=dev)
+        idx = torch.empty((w.B, w.Hq, w.n, C_max), dtype=torch.int32,
+                          device=dev)
+        cnt = torch.empty((w.B, w.Hq, w.n), dtype=torch.int32, device=dev)
+    ws = torch.empty(ca.condensate_attn_workspace_size(
+        decode, tdt, w.B, w.n, w.Hq, w.Hkv, w.d, W_max, w.k),
+        dtype=torch.uint8, device=dev)
+    fn = ca.condensate_attn_decode if decode else ca.condensate_attn_prefill
+
+    def step(qin):
+        fn(qin, K, V, w.W, w.k, W_i=W_i, O=O, idx=idx, idx_count=cnt,
+           C_max=C_max, workspace=ws)
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(Q)
+    st = ca.condensate_attn_status(ws)
+    if st != ca.CA_OK:
+        raise RuntimeError(f"device status: {ca.status_string(st)}")
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+
+    # ---- device-resident timed region
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    binding.profile_start(8 * args.steps + 16)
+    for s in range(args.steps):
+        flush.zero_()  # L2 flush, outside the step's events
+        evs[s][0].record()
+        step(Q)
+        evs[s][1].record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    prof = binding.profile_stop(8 * args.steps + 16)
+    if dist:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    if decode:
+        q_host = pin(Q)
+        q_host.copy_(Q.cpu())
+        q_dev = torch.empty_like(Q)
+        h2d = q_host.numel() * q_host.element_size()
+    else:
+        # prefill consumes Q, K and V of the step
+        hosts = [pin(t) for t in (Q, K, V)]
+        for h_, t_ in zip(hosts, (Q, K, V)):
+            h_.copy_(t_.cpu())
+        h2d = sum(h_.numel() * h_.element_size() for h_ in hosts)
+    outs = [pin(O), pin(idx), pin(cnt)]
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.zero_()
+        e2e_ev[s][0].record()
+        if decode:
+            q_dev.copy_(q_host, non_blocking=True)
+            step(q_dev)
+        else:
+            Q.copy_(hosts[0], non_blocking=True)
+            K.copy_(hosts[1], non_blocking=True)
+            V.copy_(hosts[2], non_blocking=True)
+            step(Q)
+        for o_h, o_d in zip(outs, (O, idx, cnt)):
+            o_h.copy_(o_d, non_blocking=True)
+        e2e_ev[s][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
+    clk = clocks.stop()
+    st = ca.condensate_attn_status(ws)
+    if st != ca.CA_OK:
+        raise RuntimeError(f"device status: {ca.status_string(st)}")
+
+    ms = statistics.mean(step_ms)
+    e2e_mean = statistics.mean(e2e_ms)
+    if dist:
+        tm = torch.tensor([ms, e2e_mean], device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms, e2e_mean = float(tm[0]), float(tm[1])
+
+    # per-kernel device times
+    per = {}
+    for name, t in prof:
+        per.setdefault(name, []).append(t)
+    kern_avg = {k_: statistics.mean(v) for k_, v in per.items()}
+    launches = len(prof)
+    pk = peaks()
+    model = work_model(w)
+    dom = max(kern_avg, key=lambda k_: sum(per[k_]))
+    bound, work, what = model[dom]
+    t_dom = kern_avg[dom] * 1e-3
+    if bound == "tensor":
+        achieved = work / t_dom / 1e12
+        peak, unit = pk["bf16_tflops"], "TFLOP/s"
+    elif bound == "hbm":
+        achieved = work / t_dom / 1e9
+        peak, unit = pk["hbm_gbs"], "GB/s"
+    else:
+        achieved = work / t_dom / 1e12
+        # fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock
+        peak = 148 * 128 * 2 * (clk["sm_max_mhz"] or 1965.0) * 1e6 / 1e12
+        unit = "TFLOP/s"
+    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+            "unit": unit, "frac": achieved / peak,
+            "peak_source": pk["source"] + (" burst" if bound != "alu" else
+                                           " derived"),
+            "work_per_launch": work, "work_definition": what,
+            "avg_launch_ms": kern_avg[dom],
+            "traffic": traffic_for(dom, w.name)}
+    units = step_units(w) * world
+    if decode:
+        value, unit_v, hib = ms, "ms", False
+        # whole-step HBM roofline: K scored + K/V rows of C_i gathered
+        step_bytes = (model["decode_score_topk"][1]
+                      + model["decode_merge_attend"][1])
+        step_roof = {"bytes": step_bytes,
+                     "achieved_gbs": step_bytes / (ms * 1e-3) / 1e9,
+                     "frac": step_bytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        e2e_val, e2e_unit = e2e_mean, "ms"
+    else:
+        value, unit_v, hib = units / (ms * 1e-3), "tokens/s", True
+        step_roof = {"flops": work, "achieved_tflops":
+                     model["prefill_score_topk_tc"][1] / (ms * 1e-3) / 1e12}
+        e2e_val, e2e_unit = units / (e2e_mean * 1e-3), "tokens/s"
+    out = {
+        "metric": METRIC, "value": value, "unit": unit_v, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": hib, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded; see workloads/)",
+        "config": {"workload": w.name, "description": w.description,
+                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   ("L" if decode else "n"): w.n, "W": w.W, "k": w.k,
+                   "adaptive_window": w.adaptive,
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "flushed before every step (256 MiB write), "
+                         "outside the step's events"},
+        "roofline": roof, "step_roofline": step_roof,
+        "kernels_avg_ms": kern_avg,
+        "tokens_per_s": units / (ms * 1e-3),
+        "e2e": {"value": e2e_val, "unit": e2e_unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": ("per-step query H2D (KV cache resident), call, "
+                         "O/idx/count D2H" if decode else
+                         "Q/K/V H2D, call, O/idx/count D2H")},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(w, x, budget_s=15.0)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+# ----------------------------------------------------------------- oracle
+def cpu_baseline(w, x, budget_s=15.0, seed=0):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    threads = oracle.max_threads()
+    if w.kind == "decode":
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.decode(x["Q"], x["K"], x["V"], w.W, w.k, W_i=x["W_i"],
+                          C_max=min(w.n, w.C_max), with_full=False)
+            reps += 1
+            if time.perf_counter() - t0 > budget_s or reps >= 5:
+                break
+        per = (time.perf_counter() - t0) / reps
+        return {"value": per * 1e3, "unit": "ms", "cores": threads,
+                "kind": "oracle",
+                "sample": f"{reps} full decode step(s) of {w.name} "
+                          f"(all {w.B * w.Hq} q-heads, L={w.n})"}
+    rng = np.random.default_rng(seed)
+    R = w.B * w.Hq * w.n
+    done, rows_total, t_total = 0, 0, 0.0
+    batch = 64
+    while t_total < budget_s and rows_total < R:
+        sel = np.stack([rng.integers(w.B, size=batch),
+                        rng.integers(w.Hq, size=batch),
+                        rng.integers(w.n, size=batch)], 1)
+        t0 = time.perf_counter()
+        oracle.prefill(x["Q"], x["K"], x["V"], w.W, w.k, W_i=x["W_i"],
+                       sel=sel, C_max=w.C_max, with_full=False)
+        t_total += time.perf_counter() - t0
+        rows_total += batch
+        done += 1
+    per_row = t_total / rows_total
+    return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows_total} uniformly drawn query rows of {w.name}; "
+                      f"rate extrapolated per row"}
+
+
+def run_reference(args):
+    w = workloads.get(args.workload)
+    x = workloads.generate(w)
+    vals = []
+    for s in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, x, budget_s=2.0, seed=s)
+        if s >= args.warmup:
+            vals.append(cb["value"])
+    v = statistics.mean(vals)
+    decode = w.kind == "decode"
+    cb["value"] = v
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": cb["unit"],
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": v if decode else None,
+        "higher_is_better": not decode, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; see workloads/)",
+        "config": {"workload": w.name, "description": w.description},
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": cb["unit"], "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

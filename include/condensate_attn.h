@@ -123,6 +123,19 @@ CA_API ca_status condensate_attn_status(void* workspace, void* stream);
 /* Static, human-readable name of a status code. */
 CA_API const char* condensate_attn_status_string(ca_status s);
 
+/*
+ * Per-launch timing for benchmarks (not part of the computation).  Between
+ * start and stop, every kernel the library launches is bracketed by CUDA
+ * events on its stream, up to `capacity` launches.  stop() waits for the
+ * recorded events and writes, per launch in issue order, the kernel's name
+ * (a static string) and its device time in milliseconds; returns the number
+ * of records written (at most cap).  Process-wide switch: not for use while
+ * other threads call the library.
+ */
+CA_API ca_status condensate_attn_profile_start(int capacity);
+CA_API int condensate_attn_profile_stop(const char** names, float* ms,
+                                        int cap);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 CA_API int condensate_attn_version(void);
 

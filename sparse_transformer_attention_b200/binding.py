@@ -43,6 +43,9 @@ SIGNATURES = {
     "condensate_attn_status": (_I, [_P, _P]),
     "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
     "condensate_attn_version": (_I, []),
+    "condensate_attn_profile_start": (_I, [_I]),
+    "condensate_attn_profile_stop": (_I, [ctypes.POINTER(ctypes.c_char_p),
+                                          ctypes.POINTER(ctypes.c_float), _I]),
 }
 
 _lib = None
@@ -198,3 +201,17 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
 def condensate_attn_status(workspace: torch.Tensor, stream=None) -> int:
     """Wait for the stream and return (and clear) the device status code."""
     return int(load().condensate_attn_status(_ptr(workspace), _stream(stream)))
+
+
+def profile_start(capacity: int = 4096) -> None:
+    """Start recording per-launch device times (see the header)."""
+    _check(load().condensate_attn_profile_start(int(capacity)),
+           "condensate_attn_profile_start")
+
+
+def profile_stop(cap: int = 4096):
+    """Stop recording; returns [(kernel name, milliseconds), ...]."""
+    names = (ctypes.c_char_p * cap)()
+    ms = (ctypes.c_float * cap)()
+    n = load().condensate_attn_profile_stop(names, ms, cap)
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]

@@ -17,6 +17,7 @@
 // an fp32 online softmax over the gathered K/V rows of C_i.
 #include "common.cuh"
 #include "decode.cuh"
+#include "profile.cuh"
 #include "select.cuh"
 
 namespace ca {
@@ -400,7 +401,9 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
       k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
   dim3 grid1(a.nchunks, a.Hkv, a.B);
+  prof_before(stream, "decode_score_topk");
   k1<<<grid1, kThreads, smem1, stream>>>(a);
+  prof_after(stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t smem2 = (size_t)a.nchunks * a.k * 8 + (size_t)a.kpow2 * 4 +
@@ -411,13 +414,17 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem2);
     if (e != cudaSuccess) return e;
+    prof_before(stream, "decode_merge_attend");
     k2<<<grid2, kMergeThreads, smem2, stream>>>(a);
+    prof_after(stream);
   } else {
     auto k2 = decode_merge_attend<T, D, float>;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem2);
     if (e != cudaSuccess) return e;
+    prof_before(stream, "decode_merge_attend");
     k2<<<grid2, kMergeThreads, smem2, stream>>>(a);
+    prof_after(stream);
   }
   return cudaGetLastError();
 }

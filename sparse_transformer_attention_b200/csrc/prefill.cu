@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "prefill.cuh"
+#include "profile.cuh"
 #include "row_topk.cuh"
 #include "sm100.cuh"
 
@@ -536,7 +537,9 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
+  prof_before(s, "prefill_score_topk_tc");
   kern<<<grid, 192, smem, s>>>(tq, tk, a);
+  prof_after(s);
   return cudaGetLastError();
 }
 
@@ -549,7 +552,9 @@ cudaError_t launch_select_f32(const PrefillArgs& a, cudaStream_t s) {
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
+  prof_before(s, "prefill_score_topk_f32");
   kern<<<grid, kTileRows, smem, s>>>(a);
+  prof_after(s);
   return cudaGetLastError();
 }
 
@@ -559,6 +564,7 @@ cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
   const int64_t warps = (R + 7) / 8;
   const int64_t blocks = (warps * 32 + kGatherThreads - 1) / kGatherThreads;
   dim3 grid((unsigned)blocks);
+  prof_before(s, "prefill_gather");
   if (a.k <= 32) {
     if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 1><<<grid, kGatherThreads, 0, s>>>(a);
     else prefill_gather<T, D, float, 1><<<grid, kGatherThreads, 0, s>>>(a);
@@ -566,6 +572,7 @@ cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
     if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 2><<<grid, kGatherThreads, 0, s>>>(a);
     else prefill_gather<T, D, float, 2><<<grid, kGatherThreads, 0, s>>>(a);
   }
+  prof_after(s);
   return cudaGetLastError();
 }
 
