@@ -114,6 +114,28 @@ CA_API ca_status condensate_attn_decode(const void* q, const void* K, const void
                                  void* stream);
 
 /*
+ * Decode without a workspace argument, for callers that cannot allocate
+ * device memory or pass a scratch pointer (a plugin whose host exposes no
+ * allocator, a fully pre-budgeted memory plan, a fixed interface with no
+ * scratch argument).  The paper has no counterpart to this entry point.
+ * Same arguments, results and checks as condensate_attn_decode on the
+ * current device, but the scratch comes from a 4 MiB buffer compiled into
+ * the library (held on every GPU that loads it until exit).  Problems whose
+ * decode workspace (condensate_attn_workspace_size) exceeds 4 MiB are
+ * rejected with CA_ERR_WORKSPACE before any launch.  Allocates nothing.  The
+ * first call on a device looks up the buffer's device address; make it
+ * before any stream capture.  All calls on a device share the buffer: calls
+ * that overlap on the GPU race and must be serialised by the caller.
+ * Device-side flags (W_i below 1, C_max overflow) land in the shared buffer
+ * and are not reported by this entry point.
+ */
+CA_API ca_status condensate_attn_decode_noalloc(
+    const void* q, const void* K, const void* V, ca_dtype dtype, int B, int L,
+    int Hq, int Hkv, int d, int W, int k, const int32_t* W_i, void* O,
+    ca_dtype o_dtype, int32_t* idx, int32_t* idx_count, int C_max,
+    void* stream);
+
+/*
  * Waits for `stream`, then reads and clears the device status word of
  * `workspace`: CA_OK, CA_ERR_DEVICE_ARG or CA_ERR_TIMEOUT (CA_ERR_CUDA if
  * the wait or copy itself failed).

@@ -40,6 +40,9 @@ SIGNATURES = {
     "condensate_attn_decode":
         (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
               _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_decode_noalloc":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
+              _I, _P]),
     "condensate_attn_status": (_I, [_P, _P]),
     "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
     "condensate_attn_version": (_I, []),
