@@ -234,7 +234,6 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    binding.profile_start(8 * args.steps + 16)
     for s in range(args.steps):
         flush.zero_()  # L2 flush, outside the step's events
         evs[s][0].record()
@@ -242,10 +241,18 @@ def run_ours(args, rank, world, local_rank):
         evs[s][1].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
-    prof = binding.profile_stop(8 * args.steps + 16)
     if dist:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
+    # Per-kernel device times come from a separate pass: the library's event
+    # records between its launches would otherwise serialise the dependent
+    # launch of the second kernel inside the timed steps.
+    binding.profile_start(8 * args.steps + 16)
+    for s in range(args.steps):
+        flush.zero_()
+        step(Q)
+    torch.cuda.synchronize()
+    prof = binding.profile_stop(8 * args.steps + 16)
 
     # ---- end to end through the public API with host buffers
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -298,7 +305,7 @@ def run_ours(args, rank, world, local_rank):
     for name, t in prof:
         per.setdefault(name, []).append(t)
     kern_avg = {k_: statistics.mean(v) for k_, v in per.items()}
-    launches = len(prof)
+    launches = len(prof)  # library kernels launched per timed pass
     pk = peaks()
     model = work_model(w)
     dom = max(kern_avg, key=lambda k_: sum(per[k_]))

@@ -27,7 +27,8 @@ bool group_ok(int Hq, int Hkv) {
 
 size_t decode_ws(int B, int L, int Hq, int Hkv, int k) {
   int nch = ca::decode_chunks(B, L, Hkv, k);
-  return ca::kStatusBytes + round_up((size_t)B * Hq * nch * (k > 0 ? k : 1) * 8, 256);
+  return ca::kStatusBytes +
+         round_up((size_t)B * Hq * nch * (k > 0 ? k : 1) * 8, 256);
 }
 
 }  // namespace
@@ -97,7 +98,7 @@ ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
   ca_status st = check_common(q, K, V, dtype, B, L, Hq, Hkv, d, W, k, W_i, O,
                               o_dtype, idx, idx_count, C_max, workspace);
   if (st != CA_OK) return st;
-  if (k > 4096) return CA_ERR_UNSUPPORTED;
+  if (k > ca::kDecodeMaxK) return CA_ERR_UNSUPPORTED;
   if (workspace_bytes < decode_ws(B, L, Hq, Hkv, k)) return CA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(workspace, 0, ca::kStatusBytes, s) != cudaSuccess)

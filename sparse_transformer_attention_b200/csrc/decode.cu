@@ -3,31 +3,48 @@
 // §2.1 Definition 1 (C_i for the last row), §2.2.3 (Dynamic Top-k), §2.4
 // Corollary 3 (per-query window), §5.2.2 (select, then attend on the subset).
 //
-// Launch 1, decode_score_topk: grid (chunks, Hkv, B).  Each CTA streams one
-// chunk of K rows of one kv-head once, with 16-byte coalesced loads (8 lanes
-// per 256-byte row), scores all G = Hq/Hkv q-heads of the group from the same
-// bytes, and keeps a per-head candidate buffer in shared memory behind a
-// threshold that only rises.  Buffers are cut back to exactly the best k
-// keys by a CTA radix select; the chunk's best k keys per q-head go to the
-// workspace.  The union of the chunks' best-k lists contains the global
-// Top-k, since every global Top-k member is among the best k of its chunk.
+// Launch 1, decode_score_topk: grid (chunks, Hkv, B), about two CTAs per SM.
+// One producer thread streams the chunk's contiguous K rows into a ring of
+// 16 KiB shared-memory stages with bulk asynchronous copies (no multicast),
+// so the loads stay deep in flight whatever the compute warps are doing.
+// Eight compute warps read each K row once from shared memory (8 lanes per
+// row, 16-byte reads, conflict-free), score all G = Hq/Hkv q-heads of the
+// group from the same bytes with packed fp32 FMAs, and keep a per-head
+// candidate buffer in shared memory behind a threshold that only rises.
+// Buffers are cut back to exactly the best k keys by a radix select over
+// the compute warps; the chunk's best k keys per q-head go to the workspace.
+// The union of the chunks' best-k lists contains the global Top-k, since
+// every global Top-k member is among the best k of its own chunk.
 //
-// Launch 2, decode_merge_attend: grid (Hq, B).  Each CTA merges its q-head's
-// chunk lists into the exact Top-k, writes C_i in ascending order, then runs
-// an fp32 online softmax over the gathered K/V rows of C_i.
+// Launch 2, decode_merge_attend: grid (Hq, B).  Half of each CTA gathers the
+// anchor and window rows and runs their fp32 online softmax while the other
+// half merges the chunk lists into the exact Top-k (radix select), writes
+// C_i in ascending order and accumulates the Top-k rows, whose scores come
+// with their keys; the two partial softmax states are then combined.
 #include "common.cuh"
 #include "decode.cuh"
 #include "profile.cuh"
 #include "select.cuh"
+#include "sm100.cuh"
 
 namespace ca {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSub = 1024;     // keys per sub-chunk between buffer checks
-constexpr int kSlack = 512;    // insert room kept after a cut
+constexpr int kComputeWarps = 8;
+constexpr int kCompute = kComputeWarps * 32;  // compute threads
+constexpr int kThreads = kCompute + 32;       // + one producer warp
+constexpr int kStageBytes = 16384;
+constexpr int kMaxStages = 6;  // K staging ring depth (chosen per launch)
+constexpr int kSub = 512;     // keys between candidate-buffer checks
+constexpr int kMinSlack = 256;      // smallest insert room kept after a cut
+constexpr int kMaxSlack = 2048;     // largest useful insert room
+constexpr size_t kSmemTwoCtas = 108 * 1024;   // two CTAs per SM, with margin
+constexpr size_t kSmemOneCta = 227 * 1024;
 constexpr int kMergeThreads = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per bounded wait
+using ComputeBar = GroupBarrier<1, kCompute>;
+using MergeBar = GroupBarrier<1, 256>;
 
 // Transposing butterfly over the 8 lanes of one key.  On entry v[h] is this
 // lane's partial dot product for q-head h of the group; every step halves
@@ -75,244 +92,553 @@ __device__ __forceinline__ bool reduce_owner(int l8) {
 
 template <int G>
 struct TopkShared {
-  int cnt[G];
-  int kk[G];
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t thr[G];
-  uint64_t T[G];
-  int out_pos;
-  SelectState<G> sel;
+  int cnt[G];
+  int abort;
+  uint32_t hist[G][256];  // one radix histogram per list (per cutting warp)
 };
 
-// Cut every list whose count exceeds `limit` down to its best k keys.
-template <int G>
-__device__ void cut_lists(uint64_t* buf, int cap, uint64_t* tmp, int k,
-                          int limit, TopkShared<G>* sh) {
-  __shared__ int s_n[G];
-  bool any = false;
-#pragma unroll
-  for (int h = 0; h < G; ++h) any = any || (sh->cnt[h] > limit);
-  if (!any) return;  // uniform decision
-  if (threadIdx.x < G) {
-    s_n[threadIdx.x] = sh->cnt[threadIdx.x] > limit ? sh->cnt[threadIdx.x] : 0;
-    sh->kk[threadIdx.x] = k;
+// Bounded wait on a stage barrier; a time-out raises the CTA's abort flag
+// (and the status bit) so that every other wait returns at once.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity,
+                                           volatile int* abort_flag,
+                                           uint32_t* status) {
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (true) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (sm100::globaltimer_ns() - t0 > kWaitNs) {
+      *abort_flag = 1;
+      raise_flag(status, kErrTimeout);
+      return false;
+    }
   }
-  __syncthreads();
-  cta_select_thresholds<kThreads, G>(buf, cap, s_n, sh->kk, sh->T, &sh->sel);
+}
+
+// One warp cuts the list lst[0..n) of unique keys down to its best kk keys
+// (n > kk >= 1), in place and in no particular order, and returns the
+// threshold T with exactly kk keys >= T.  Radix select from the most
+// significant byte, stopping as soon as the chosen byte's bucket holds
+// exactly the keys still needed (its lower bound then separates the sets).
+__device__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint32_t* hist,
+                             int lane) {
+  uint64_t prefix = 0ull;
+  uint32_t need = (uint32_t)kk;
 #pragma unroll 1
-  for (int h = 0; h < G; ++h) {
-    if (s_n[h] == 0) continue;
-    const uint64_t T = sh->T[h];
-    if (threadIdx.x == 0) sh->out_pos = 0;
-    __syncthreads();
-    for (int e = threadIdx.x; e < s_n[h]; e += kThreads) {
-      uint64_t key = buf[h * cap + e];
-      if (key >= T) tmp[atomicAdd(&sh->out_pos, 1)] = key;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    const uint64_t hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
+#pragma unroll
+    for (int b = lane; b < 256; b += 32) hist[b] = 0u;
+    __syncwarp();
+    for (int e = lane; e < n; e += 32) {
+      const uint64_t key = lst[e];
+      if ((key & hmask) == prefix)
+        atomicAdd(&hist[(uint32_t)(key >> shift) & 255u], 1u);
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < k; e += kThreads) buf[h * cap + e] = tmp[e];
-    if (threadIdx.x == 0) {
-      sh->cnt[h] = k;
-      sh->thr[h] = T;
+    __syncwarp();
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      c[t] = hist[255 - 8 * lane - t];
+      sum += c[t];
     }
-    __syncthreads();
+    uint32_t incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const bool mine = excl < need && need <= incl;
+    uint32_t digit = 0, nd = 0, bucket = 0;
+    if (mine) {
+      uint32_t acc = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (acc + c[t] >= need) {
+          digit = 255u - 8u * lane - t;
+          nd = need - acc;
+          bucket = c[t];
+          break;
+        }
+        acc += c[t];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
+    nd = __shfl_sync(0xFFFFFFFFu, nd, src);
+    bucket = __shfl_sync(0xFFFFFFFFu, bucket, src);
+    prefix |= (uint64_t)digit << shift;
+    need = nd;
+    __syncwarp();  // the histogram is cleared again next pass
+    if (bucket == nd) break;
   }
+  // keep the keys >= prefix, packed to the front in reading order; a slot
+  // is only written after the whole group of 32 that covers it was read
+  int wr = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int e = base + lane;
+    const uint64_t key = e < n ? lst[e] : 0ull;
+    const bool keep = e < n && key >= prefix;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) lst[wr + __popc(bal & ((1u << lane) - 1u))] = key;
+    wr += __popc(bal);
+    __syncwarp();
+  }
+  return prefix;
+}
+
+// At a check point (all inserts of the stretch done): warp h cuts list h
+// when it holds more than `limit` keys.  Barriers on both sides keep every
+// compute warp from inserting while a list is being cut.
+template <int G>
+__device__ __forceinline__ void check_lists(uint64_t* buf, int cap, int k,
+                                            int limit, TopkShared<G>* sh,
+                                            int warp, int lane) {
+  ComputeBar::sync();
+  if (warp < G) {
+    const int n = sh->cnt[warp];
+    if (n > limit && n > k) {
+      const uint64_t T = warp_cut(buf + (size_t)warp * cap, n, k,
+                                  sh->hist[warp], lane);
+      if (lane == 0) {
+        sh->cnt[warp] = k;
+        sh->thr[warp] = T;
+      }
+    }
+  }
+  ComputeBar::sync();
+}
+
+template <typename T, int D, int G>
+struct ScoreCfg {
+  static constexpr int VEC = Elem<T>::kPer16B;   // elements per 16 bytes
+  static constexpr int ROWB = D * (int)sizeof(T);
+  static constexpr int CPL = ROWB / 16 / 8;       // 16-byte pieces per lane
+  static constexpr int PPL = CPL * VEC / 2;       // element pairs per lane
+  static constexpr int R = kStageBytes / ROWB;    // K rows per stage
+  static constexpr int KPR = 4 * kComputeWarps;   // keys per round
+  static constexpr int ROUNDS = R / KPR;
+  static constexpr int SUB_ST = kSub / R;         // stages per buffer check
+  static_assert(CPL >= 1 && R % KPR == 0 && kSub % R == 0, "tiling");
+};
+
+// Unpack one 16-byte piece into element pairs.
+template <typename T>
+__device__ __forceinline__ void pairs16(const uint4& v, float2* p);
+template <>
+__device__ __forceinline__ void pairs16<__nv_bfloat16>(const uint4& v,
+                                                       float2* p) {
+  p[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+  p[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+  p[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+  p[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+}
+template <>
+__device__ __forceinline__ void pairs16<float>(const uint4& v, float2* p) {
+  p[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+  p[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
 }
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, G >= 8 ? 1 : 2)
 decode_score_topk(DecodeArgs a) {
-  constexpr int VEC = Elem<T>::kPer16B;
-  constexpr int CPL = D / VEC / 8;  // 16-byte pieces per lane
-  constexpr int DPL = CPL * VEC;    // head dims per lane
-  constexpr int U = 4;              // keys in flight per lane
-  static_assert(CPL >= 1, "row too short for 8 lanes");
-
-  extern __shared__ __align__(16) unsigned char smem[];
+  using C = ScoreCfg<T, D, G>;
+  constexpr int VEC = C::VEC, CPL = C::CPL, PPL = C::PPL, R = C::R;
+  extern __shared__ __align__(128) unsigned char smem[];
   const int k = a.k;
-  const int cap = k + kSub + kSlack;
-  uint64_t* buf = reinterpret_cast<uint64_t*>(smem);  // [G][cap]
-  uint64_t* tmp = buf + (size_t)G * cap;               // [k]
-  TopkShared<G>* sh = reinterpret_cast<TopkShared<G>*>(tmp + k);
+  const int cap = a.cap;  // per-list buffer: k + kSub + slack keys
+  const int kStages = a.nstages;
+  unsigned char* stages = smem;                                  // ring
+  uint64_t* buf = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * kStageBytes);
+  TopkShared<G>* sh = reinterpret_cast<TopkShared<G>*>(buf + (size_t)G * cap);
 
+  // Let the merge kernel (launched as a programmatic dependent) start its
+  // independent prologue on SMs this grid releases.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int l8 = lane & 7, ks = lane >> 3;
-  const int64_t L = a.L;
-  const int Wb = row_window(a.W_i, b, a.W, (int)L, a.status,
+  const int L = a.L;  // positions fit in 31 bits (int L in the ABI)
+  const int Wb = row_window(a.W_i, b, a.W, L, a.status,
                             chunk == 0 && g == 0 && tid == 0);
-  const int64_t hi = (L - 1) - Wb;  // last candidate position
+  const int hi = (L - 1) - Wb;  // last candidate position
+  const int j0 = chunk * a.chunk_len;
+  const int c0 = j0 < 1 ? 1 : j0;
+  const int c1 = (j0 + a.chunk_len < hi + 1) ? j0 + a.chunk_len : hi + 1;
+  const int nrows = c1 > c0 ? c1 - c0 : 0;
+  const int nst = (nrows + R - 1) / R;
+  const T* Kg = reinterpret_cast<const T*>(a.K) +
+                ((size_t)b * a.Hkv + g) * (size_t)L * D;
 
-  // this lane's slice of the G queries, as fp32
-  float qf[G][DPL];
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&sh->full[s], 1);
+      sm100::mbar_init(&sh->empty[s], kComputeWarps);
+    }
+    for (int h = 0; h < G; ++h) {
+      sh->cnt[h] = 0;
+      sh->thr[h] = 0ull;
+    }
+    sh->abort = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &sh->abort;
+
+  if (warp == kComputeWarps) {
+    // ------------------------------------------------ producer
+    if (lane == 0 && nst > 0) {
+      int issued = 0;
+      int s = 0;
+      uint32_t ph = 0;  // parity of the ring pass of stage s
+      for (int t = 0; t < nst; ++t) {
+        if (t >= kStages &&
+            !stage_wait(&sh->empty[s], ph ^ 1, abort_flag, a.status))
+          break;
+        const int r0 = c0 + t * R;
+        const int left = nrows - t * R;
+        const int rows = left < R ? left : R;
+        const uint32_t bytes = (uint32_t)rows * C::ROWB;
+        sm100::mbar_arrive_expect_tx(&sh->full[s], bytes);
+        sm100::bulk_load(stages + s * kStageBytes, Kg + (size_t)r0 * D, bytes,
+                         &sh->full[s]);
+        issued = t + 1;
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+      // every copy this thread started must land before the CTA exits
+      for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
+        sm100::mbar_wait(&sh->full[t % kStages], (t / kStages) & 1, kWaitNs);
+    }
+    return;
+  }
+
+  // -------------------------------------------------- compute warps
+  const int l8 = lane & 7, ks = lane >> 3;
+  float2 q2[G][PPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const T* qh = reinterpret_cast<const T*>(a.q) +
                   ((size_t)b * a.Hq + (size_t)g * G + h) * D;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
-      uint4 v = *reinterpret_cast<const uint4*>(qh + (l8 + 8 * c) * VEC);
-      Elem<T>::unpack(v, &qf[h][c * VEC]);
+      const uint4 v = *reinterpret_cast<const uint4*>(qh + (l8 + 8 * c) * VEC);
+      pairs16<T>(v, &q2[h][c * (VEC / 2)]);
     }
   }
-  if (tid < G) {
-    sh->cnt[tid] = 0;
-    sh->thr[tid] = 0ull;
-  }
-  __syncthreads();
-
   const int myh = reduce_head<G>(l8);
   const bool owner = reduce_owner<G>(l8);
-  const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * L * D;
-  const int64_t j0 = (int64_t)chunk * a.chunk_len;
-  const int64_t c0 = j0 < 1 ? 1 : j0;
-  int64_t c1 = j0 + a.chunk_len;
-  if (c1 > hi + 1) c1 = hi + 1;
-  bool first_cut = true;
+  uint64_t thr = 0ull;       // admission threshold key (0: admit all)
+  float thr_f = -INFINITY;   // its score, for a cheap float pre-filter
+  const int first_keys = nrows < kSub ? nrows : kSub;
 
+  int s = 0;
+  uint32_t ph = 0;  // parity of the ring pass of stage s
 #pragma unroll 1
-  for (int64_t sub = c0; sub < c1; sub += kSub) {
-    const uint64_t thr = sh->thr[myh];
-    const int64_t wbase = sub + warp * (kSub / 8);
-#pragma unroll 1
-    for (int it = 0; it < kSub / 8; it += 4 * U) {
-      uint4 raw[U][CPL];
-      int64_t jj[U];
+  for (int t = 0; t < nst; ++t) {
+    if (t % C::SUB_ST == 0) {
+      thr = sh->thr[myh];
+      thr_f = thr ? key_score(thr) : -INFINITY;
+    }
+    const bool ok = __all_sync(
+        0xFFFFFFFFu, stage_wait(&sh->full[s], ph, abort_flag, a.status));
+    if (ok) {
+      const unsigned char* st = stages + s * kStageBytes;
+      const int rbase = c0 + t * R;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        jj[u] = wbase + it + u * 4 + ks;
-        int64_t jr = jj[u] < c1 ? jj[u] : c0;  // stay inside the row range
-        const T* row = Kg + (size_t)jr * D;
+      for (int rd = 0; rd < C::ROUNDS; ++rd) {
+        const int rloc = rd * C::KPR + warp * 4 + ks;
+        const int j = rbase + rloc;
+        uint4 piece[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c)
-          raw[u][c] = ld_stream_v4(row + (l8 + 8 * c) * VEC);
-      }
+          piece[c] = *reinterpret_cast<const uint4*>(st + rloc * C::ROWB +
+                                                     (l8 + 8 * c) * 16);
+        float2 acc[G];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float part[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) part[h] = 0.f;
+        for (int h = 0; h < G; ++h) acc[h] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
-          float f[VEC];
-          Elem<T>::unpack(raw[u][c], f);
+          float2 kp[VEC / 2];
+          pairs16<T>(piece[c], kp);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e)
+          for (int p = 0; p < VEC / 2; ++p)
 #pragma unroll
             for (int h = 0; h < G; ++h)
-              part[h] = fmaf(qf[h][c * VEC + e], f[e], part[h]);
+              acc[h] = __ffma2_rn(q2[h][c * (VEC / 2) + p], kp[p], acc[h]);
         }
-        const float s = group_reduce<G>(part, lane);
-        if (owner && jj[u] < c1) {
-          const uint64_t key = make_key(s, (uint32_t)jj[u]);
-          if (key > thr) {
-            int pos = atomicAdd(&sh->cnt[myh], 1);
-            buf[(size_t)myh * cap + pos] = key;
+        float part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] = acc[h].x + acc[h].y;
+        const float sc = group_reduce<G>(part, lane);
+        if (t < C::SUB_ST) {
+          // first stretch: every key goes in, at its own slot
+          if (owner && j < c1)
+            buf[(size_t)myh * cap + (j - c0)] = make_key(sc, (uint32_t)j);
+        } else {
+          // rare once a threshold exists: one warp vote keeps the common
+          // path flat
+          const bool cand = owner && j < c1 && sc >= thr_f;
+          if (__any_sync(0xFFFFFFFFu, cand) && cand) {
+            const uint64_t key = make_key(sc, (uint32_t)j);
+            if (key > thr) {
+              const int pos = atomicAdd(&sh->cnt[myh], 1);
+              buf[(size_t)myh * cap + pos] = key;
+            }
           }
         }
       }
     }
-    __syncthreads();
-    // The first cut sets a useful threshold; later cuts only keep room for
-    // the next sub-chunk.
-    cut_lists<G>(buf, cap, tmp, k, first_cut ? k : cap - kSub, sh);
-    first_cut = false;
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(&sh->empty[s]);
+    if (++s == kStages) {
+      s = 0;
+      ph ^= 1;
+    }
+    if (t % C::SUB_ST == C::SUB_ST - 1 || t == nst - 1) {
+      if (t < C::SUB_ST) {
+        // the first stretch filled slots 0..first_keys-1 of every list
+        ComputeBar::sync();
+        if (tid < G) sh->cnt[tid] = first_keys;
+      }
+      // the first cut sets a useful threshold; later cuts keep room for the
+      // next stretch of keys
+      check_lists<G>(buf, cap, k, t < C::SUB_ST ? k : cap - kSub, sh, warp,
+                     lane);
+    }
   }
-  __syncthreads();
-  cut_lists<G>(buf, cap, tmp, k, k, sh);
+  check_lists<G>(buf, cap, k, k, sh, warp, lane);
 
   // write this chunk's best keys per q-head; empty slots get key 0
 #pragma unroll 1
   for (int h = 0; h < G; ++h) {
-    uint64_t* out = a.cand +
-        (((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + chunk) * k;
+    const size_t lst = ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + chunk;
+    uint64_t* out = a.cand + lst * k;
     const int cnt = sh->cnt[h];
-    for (int e = tid; e < k; e += kThreads)
+    for (int e = tid; e < k; e += kCompute)
       out[e] = e < cnt ? buf[(size_t)h * cap + e] : 0ull;
   }
 }
 
-// Bitonic sort (ascending) of n_pow2 uint32 values in shared memory.
-__device__ void cta_sort_u32(uint32_t* v, int n_pow2) {
-  for (int size = 2; size <= n_pow2; size <<= 1) {
+// Ascending bitonic sort of 32*NPL values held by one warp (element
+// e = t*32 + lane in v[t]); pairs closer than 32 are exchanged by shuffles.
+template <int NPL>
+__device__ __forceinline__ void warp_bitonic(uint32_t (&v)[NPL], int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32 * NPL; size <<= 1) {
+#pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int t = threadIdx.x; t < n_pow2 / 2; t += blockDim.x) {
-        int lo = 2 * t - (t & (stride - 1));
-        int hi2 = lo + stride;
-        bool up = ((lo & size) == 0);
-        uint32_t x = v[lo], y = v[hi2];
-        if ((x > y) == up) {
-          v[lo] = y;
-          v[hi2] = x;
-        }
+      uint32_t nv[NPL];
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) {
+        const int e = t * 32 + lane;
+        const uint32_t other = (stride >= 32)
+            ? v[t ^ (stride >> 5)]
+            : __shfl_xor_sync(0xFFFFFFFFu, v[t], stride);
+        const bool up = (e & size) == 0, lower = (e & stride) == 0;
+        nv[t] = (lower == up) ? min(v[t], other) : max(v[t], other);
       }
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) v[t] = nv[t];
     }
   }
-  __syncthreads();
 }
+
+template <int NPL>
+__device__ __forceinline__ void warp_sort_n(uint32_t* a, int n, int lane) {
+  uint32_t v[NPL];
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    const int e = t * 32 + lane;
+    v[t] = e < n ? a[e] : 0xFFFFFFFFu;
+  }
+  warp_bitonic<NPL>(v, lane);
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) a[t * 32 + lane] = v[t];
+}
+
+// Sort a[0..n) ascending with one warp; a has room for kpow2 >= n entries
+// (kpow2 a power of two <= 1024); entries n..kpow2 become 0xFFFFFFFF.
+__device__ __forceinline__ void warp_sort_prefix(uint32_t* a, int n, int kpow2,
+                                                 int lane) {
+  if (kpow2 <= 32) warp_sort_n<1>(a, n, lane);
+  else if (kpow2 <= 64) warp_sort_n<2>(a, n, lane);
+  else if (kpow2 <= 128) warp_sort_n<4>(a, n, lane);
+  else if (kpow2 <= 256) warp_sort_n<8>(a, n, lane);
+  else if (kpow2 <= 512) warp_sort_n<16>(a, n, lane);
+  else warp_sort_n<32>(a, n, lane);
+}
+
+// Online-softmax state of one warp: running max m (log2 domain), sum l and
+// the lane's DL output dims.
+template <int DL>
+struct Online {
+  float m = -INFINITY, l = 0.f, o[DL];
+  __device__ __forceinline__ Online() {
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[e] = 0.f;
+  }
+  __device__ __forceinline__ void add(float s, const float* v) {
+    const float mn = fmaxf(m, s);
+    const float corr = exp2f(m - mn);
+    const float p = exp2f(s - mn);
+    l = l * corr + p;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[e] = fmaf(p, v[e], o[e] * corr);
+    m = mn;
+  }
+};
 
 template <typename T, int D, typename TO>
 __global__ void __launch_bounds__(kMergeThreads)
 decode_merge_attend(DecodeArgs a) {
-  constexpr int DL = D / 32;  // head dims per lane in the gather
+  constexpr int DL = D / 32;  // head dims per lane in the gathers
   constexpr int NW = kMergeThreads / 32;
-  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int UG = 4;       // rows in flight per warp
+  extern __shared__ __align__(128) unsigned char smem[];
   const int k = a.k;
   const int ncand = a.nchunks * k;
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem);   // [ncand]
-  uint32_t* topj = reinterpret_cast<uint32_t*>(cand + ncand);  // [kpow2]
-  SelectState<1>* st = reinterpret_cast<SelectState<1>*>(topj + a.kpow2);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem);           // [ncand]
+  uint32_t* topj = reinterpret_cast<uint32_t*>(cand + ncand);   // [kpow2]
+  float* tops = reinterpret_cast<float*>(topj + a.kpow2);       // [kpow2]
+  SelectState<1>* st = reinterpret_cast<SelectState<1>*>(tops + a.kpow2);
   __shared__ int s_n, s_kk, s_m;
   __shared__ uint64_t s_T;
-  __shared__ float s_m_w[NW], s_l_w[NW];
-  __shared__ float s_o_w[NW][D];
+  __shared__ float s_mw[NW], s_lw[NW];
+  __shared__ float s_ow[NW][D];
 
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
+  const int gtid = tid & 255, gw = warp & 7;
   const int g = h / (a.Hq / a.Hkv);
   const int64_t L = a.L, i = L - 1;
   const int Wb = row_window(a.W_i, b, a.W, (int)L, a.status, false);
   const int64_t lo = (i - Wb + 1) > 0 ? (i - Wb + 1) : 0;
   const int64_t ncand_pos = (i - Wb) > 0 ? (i - Wb) : 0;  // |[1, i-W]|
   const int m = (int)(k < ncand_pos ? k : ncand_pos);
+  const int anc = lo > 0 ? 1 : 0;
+  const int64_t count = anc + m + (i - lo + 1);
 
-  // 1. gather the chunk lists (dropping empty slots)
-  if (tid == 0) s_n = 0;
-  __syncthreads();
-  const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
-  for (int e = tid; e < ncand; e += kMergeThreads) {
-    uint64_t key = src[e];
-    if (key != 0ull) cand[atomicAdd(&s_n, 1)] = key;
-  }
-  __syncthreads();
-  // 2. exact Top-m of the union
-  if (tid == 0) s_kk = m > 0 ? m : 1;
-  __syncthreads();
-  cta_select_thresholds<kMergeThreads, 1>(cand, 0, &s_n, &s_kk, &s_T, st);
-  if (tid == 0) s_m = 0;
-  for (int e = tid; e < a.kpow2; e += kMergeThreads) topj[e] = 0xFFFFFFFFu;
-  __syncthreads();
-  if (m > 0) {
-    for (int e = tid; e < s_n; e += kMergeThreads) {
-      uint64_t key = cand[e];
-      if (key >= s_T) {
-        const uint32_t j = key_index(key);
-        const int p = atomicAdd(&s_m, 1);
-        if (p < a.kpow2 && j >= 1 && (int64_t)j <= i - Wb) topj[p] = j;
-        else raise_flag(a.status, kErrInternal);
+  const T* qh = reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + h) * D;
+  float qv[DL];
+  load_f32<T, DL>(qh + lane * DL, qv);
+  const T* Kg = reinterpret_cast<const T*>(a.K) +
+                ((size_t)b * a.Hkv + g) * (size_t)L * D + lane * DL;
+  const T* Vg = reinterpret_cast<const T*>(a.V) +
+                ((size_t)b * a.Hkv + g) * (size_t)L * D + lane * DL;
+  const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e)/sqrt(d)
+  Online<DL> acc;
+
+  if (warp >= 8) {
+    // ---------------- anchor and window rows (no dependence on selection)
+    const int64_t nwin = anc + (i - lo + 1);
+#pragma unroll 1
+    for (int64_t e0 = gw; e0 < nwin; e0 += 8 * UG) {
+      float kf[UG][DL], vf[UG][DL];
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        const int64_t e = e0 + 8 * u;
+        int64_t j = 0;
+        if (e < nwin) j = (anc && e == 0) ? 0 : lo + (e - anc);
+        load_f32<T, DL>(Kg + (size_t)j * D, kf[u]);
+        load_f32<T, DL>(Vg + (size_t)j * D, vf[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        if (e0 + 8 * u >= nwin) break;  // warp-uniform
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) dot = fmaf(qv[e], kf[u][e], dot);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
+        acc.add(dot * sl2, vf[u]);
+      }
+    }
+  } else {
+    // ---------------- merge the chunk lists into the exact Top-k
+    // The lists are written by the score kernel, which may still be
+    // finishing: wait for it (programmatic dependent launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (gtid == 0) {
+      s_n = 0;
+      s_m = 0;
+      s_kk = m > 0 ? m : 1;
+    }
+    MergeBar::sync();
+    const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
+    for (int e = gtid; e < ncand; e += 256) {
+      const uint64_t key = src[e];
+      if (key != 0ull) cand[atomicAdd(&s_n, 1)] = key;
+    }
+    MergeBar::sync();
+    cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
+                                            gtid);
+    if (m > 0) {
+      for (int e = gtid; e < s_n; e += 256) {
+        const uint64_t key = cand[e];
+        if (key >= s_T) {
+          const uint32_t j = key_index(key);
+          const int p = atomicAdd(&s_m, 1);
+          if (p < m && j >= 1 && (int64_t)j <= i - Wb) {
+            topj[p] = j;
+            tops[p] = key_score(key);
+          } else {
+            raise_flag(a.status, kErrInternal);
+          }
+        }
       }
     }
   }
   __syncthreads();
+  const int got = s_m < m ? s_m : m;
   if (m > 0 && s_m != m && tid == 0) raise_flag(a.status, kErrInternal);
-  // an inconsistent candidate list must never steer the gather out of range
-  for (int e = tid; e < a.kpow2; e += kMergeThreads)
-    if (e >= m || topj[e] == 0xFFFFFFFFu) topj[e] = e < m ? 0u : 0xFFFFFFFFu;
-  cta_sort_u32(topj, a.kpow2);
-
-  // 3. C_i = {0} U sorted Top-k U [lo, i], ascending
-  const int anc = lo > 0 ? 1 : 0;
-  const int64_t count = anc + m + (i - lo + 1);
+  // Top-k rows, spread over all warps: the score travels with the key, so
+  // only V is read
+#pragma unroll 1
+  for (int e0 = warp; e0 < got; e0 += NW * UG) {
+    float vf[UG][DL];
+#pragma unroll
+    for (int u = 0; u < UG; ++u) {
+      const int e = e0 + NW * u;
+      const uint32_t j = e < got ? topj[e] : 0u;
+      load_f32<T, DL>(Vg + (size_t)j * D, vf[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < UG; ++u) {
+      const int e = e0 + NW * u;
+      if (e >= got) break;  // warp-uniform
+      acc.add(tops[e] * sl2, vf[u]);
+    }
+  }
+  if (lane == 0) {
+    s_mw[warp] = acc.m;
+    s_lw[warp] = acc.l;
+  }
+#pragma unroll
+  for (int e = 0; e < DL; ++e) s_ow[warp][lane * DL + e] = acc.o[e];
+  __syncthreads();  // every warp is done reading topj
+  // C_i = {0} U sorted Top-k U [lo, i], ascending, for the idx output
+  if (warp == 0) warp_sort_prefix(topj, got, a.kpow2, lane);
+  if (tid >= 32 && tid < 32 + D) {
+    const int dd = tid - 32;
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_mw[w]);
+    float l = 0.f, o = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      if (s_lw[w] == 0.f) continue;
+      const float c = exp2f(s_mw[w] - M);
+      l += s_lw[w] * c;
+      o += s_ow[w][dd] * c;
+    }
+    TO* out = reinterpret_cast<TO*>(a.O) + ((size_t)b * a.Hq + h) * D;
+    store_out<TO>(out + dd, o / l);
+  }
+  __syncthreads();  // the sorted Top-k is visible
   int32_t* idx_row = a.idx + ((size_t)b * a.Hq + h) * a.C_max;
   if (count > a.C_max && tid == 0) raise_flag(a.status, kErrCmax);
   const int64_t wcount = count < a.C_max ? count : a.C_max;
@@ -320,112 +646,84 @@ decode_merge_attend(DecodeArgs a) {
     int32_t v;
     if (r >= wcount) v = -1;
     else if (r < anc) v = 0;
-    else if (r < anc + m) v = (int32_t)topj[r - anc];
+    else if (r < anc + m) v = (r - anc < got) ? (int32_t)topj[r - anc] : 0;
     else v = (int32_t)(lo + (r - anc - m));
     idx_row[r] = v;
   }
   if (tid == 0) a.idx_count[(size_t)b * a.Hq + h] = (int32_t)count;
+}
 
-  // 4. fp32 online softmax over C_i; warps take entries r = warp + NW*t,
-  //    lanes split the head dimension.
-  const T* qh = reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + h) * D;
-  float qv[DL];
-  load_f32<T, DL>(qh + lane * DL, qv);
-  const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * L * D;
-  const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * L * D;
-  const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e)/sqrt(d)
-  float mx = -INFINITY, den = 0.f, o[DL];
-#pragma unroll
-  for (int e = 0; e < DL; ++e) o[e] = 0.f;
-  constexpr int UG = 4;  // entries in flight per warp
-#pragma unroll 1
-  for (int64_t r0 = warp; r0 < count; r0 += NW * UG) {
-    float kf[UG][DL], vf[UG][DL];
-#pragma unroll
-    for (int u = 0; u < UG; ++u) {
-      const int64_t r = r0 + (int64_t)NW * u;
-      int64_t j = 0;
-      if (r < anc) j = 0;
-      else if (r < anc + m) j = topj[r - anc];
-      else if (r < count) j = lo + (r - anc - m);
-      load_f32<T, DL>(Kg + (size_t)j * D + lane * DL, kf[u]);
-      load_f32<T, DL>(Vg + (size_t)j * D + lane * DL, vf[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < UG; ++u) {
-      if (r0 + (int64_t)NW * u >= count) break;  // warp-uniform
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < DL; ++e) dot = fmaf(qv[e], kf[u][e], dot);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-        dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
-      const float s = dot * sl2;
-      const float mn = fmaxf(mx, s);
-      const float corr = exp2f(mx - mn);
-      const float p = exp2f(s - mn);
-      den = den * corr + p;
-#pragma unroll
-      for (int e = 0; e < DL; ++e) o[e] = fmaf(p, vf[u][e], o[e] * corr);
-      mx = mn;
-    }
-  }
-  if (lane == 0) {
-    s_m_w[warp] = mx;
-    s_l_w[warp] = den;
-  }
-#pragma unroll
-  for (int e = 0; e < DL; ++e) s_o_w[warp][lane * DL + e] = o[e];
-  __syncthreads();
-  if (tid < D) {
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m_w[w]);
-    float l = 0.f, acc = 0.f;
-    for (int w = 0; w < NW; ++w) {
-      if (s_l_w[w] == 0.f) continue;
-      const float c = exp2f(s_m_w[w] - M);
-      l += s_l_w[w] * c;
-      acc += s_o_w[w][tid] * c;
-    }
-    TO* out = reinterpret_cast<TO*>(a.O) + ((size_t)b * a.Hq + h) * D;
-    store_out<TO>(out + tid, acc / l);
-  }
+
+// Shared memory of the score kernel: a K staging ring of 3..kMaxStages
+// stages and per-list candidate buffers of k + kSub + slack keys.  Prefer
+// two CTAs per SM; spend what is left after the ring on insert slack.
+template <int G>
+void score_smem(int k, int* cap, int* nstages, size_t* bytes) {
+  const size_t fixed = sizeof(TopkShared<G>);
+  const size_t min_lists = (size_t)G * 8 * (k + kSub + kMinSlack);
+  size_t budget = kSmemTwoCtas;
+  if (fixed + min_lists + 3 * (size_t)kStageBytes > budget) budget = kSmemOneCta;
+  // Three stages keep the stream fed (deeper rings measured no faster);
+  // the rest goes to insert slack, which makes list cuts rarer.
+  long st = budget == kSmemTwoCtas
+                ? 3
+                : (long)((budget - fixed - min_lists) / kStageBytes);
+  if (st > kMaxStages) st = kMaxStages;
+  if (st < 2) st = 2;
+  const size_t rem = budget - fixed - (size_t)st * kStageBytes;
+  long slack = (long)(rem / (8 * G)) - k - kSub;
+  if (slack > kMaxSlack) slack = kMaxSlack;
+  if (slack < kMinSlack) slack = kMinSlack;
+  *cap = k + kSub + (int)slack;
+  *nstages = (int)st;
+  *bytes = (size_t)st * kStageBytes + (size_t)G * 8 * (size_t)(*cap) + fixed;
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
-  const int cap = a.k + kSub + kSlack;
-  size_t smem1 = (size_t)G * cap * 8 + (size_t)a.k * 8 + sizeof(TopkShared<G>);
-  auto k1 = decode_score_topk<T, D, G>;
-  cudaError_t e = cudaFuncSetAttribute(
-      k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-  if (e != cudaSuccess) return e;
-  dim3 grid1(a.nchunks, a.Hkv, a.B);
-  prof_before(stream, "decode_score_topk");
-  k1<<<grid1, kThreads, smem1, stream>>>(a);
-  prof_after(stream);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  size_t smem2 = (size_t)a.nchunks * a.k * 8 + (size_t)a.kpow2 * 4 +
-                 sizeof(SelectState<1>);
-  dim3 grid2(a.Hq, a.B);
-  if (a.o_bf16) {
-    auto k2 = decode_merge_attend<T, D, __nv_bfloat16>;
-    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem2);
+cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
+  size_t smem1;
+  score_smem<G>(a.k, &a.cap, &a.nstages, &smem1);
+  cudaError_t e = cudaSuccess;
+  if (a.k > 0) {  // with k = 0 the set is anchor and window only
+      auto k1 = decode_score_topk<T, D, G>;
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem1);
     if (e != cudaSuccess) return e;
-    prof_before(stream, "decode_merge_attend");
-    k2<<<grid2, kMergeThreads, smem2, stream>>>(a);
-    prof_after(stream);
-  } else {
-    auto k2 = decode_merge_attend<T, D, float>;
-    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem2);
+    // ask for the largest shared-memory carve-out so two CTAs fit per SM
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    prof_before(stream, "decode_merge_attend");
-    k2<<<grid2, kMergeThreads, smem2, stream>>>(a);
+    dim3 grid1(a.nchunks, a.Hkv, a.B);
+    prof_before(stream, "decode_score_topk");
+    k1<<<grid1, kThreads, smem1, stream>>>(a);
     prof_after(stream);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
+  const size_t smem2 = (size_t)a.nchunks * a.k * 8 + (size_t)a.kpow2 * 8 +
+                       sizeof(SelectState<1>);
+  dim3 grid2(a.Hq, a.B);
+  auto k2 = a.o_bf16 ? decode_merge_attend<T, D, __nv_bfloat16>
+                     : decode_merge_attend<T, D, float>;
+  e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem2);
+  if (e != cudaSuccess) return e;
+  // Programmatic dependent launch: the merge grid may start while the score
+  // grid drains; it waits (griddepcontrol.wait) before reading the lists.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid2;
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = smem2;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  prof_before(stream, "decode_merge_attend");
+  e = cudaLaunchKernelEx(&cfg, k2, a);
+  prof_after(stream);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -8,6 +8,9 @@ namespace ca {
 
 // About two CTAs per SM on a 148-SM B200 for the K-streaming pass.
 constexpr int kDecodeTargetCtas = 296;
+// Largest Top-k of the decode path (the per-head candidate buffers of the
+// score pass must fit in shared memory next to the K staging ring).
+constexpr int kDecodeMaxK = 1024;
 // Upper bound on merged candidates per q-head (chunks x k), so the merge
 // fits in shared memory.
 constexpr int kDecodeMaxMerge = 8192;
@@ -24,7 +27,9 @@ struct DecodeArgs {
   int32_t* idx_count;
   int C_max;
   int chunk_len, nchunks, kpow2;
-  uint64_t* cand;     // [B, Hq, nchunks, k] chunk-best keys (workspace)
+  int cap;              // per-list candidate buffer of the score kernel
+  int nstages;          // K staging ring depth of the score kernel
+  uint64_t* cand;       // [B, Hq, nchunks, k] chunk-best keys (workspace)
   uint32_t* status;   // device status word (workspace)
 };
 

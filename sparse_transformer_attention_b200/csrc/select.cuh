@@ -13,6 +13,18 @@
 
 namespace ca {
 
+// Barrier policies: the whole CTA, or a named barrier over the N threads of
+// one warp group (the other warps of the CTA keep running).
+struct CtaBarrier {
+  __device__ static __forceinline__ void sync() { __syncthreads(); }
+};
+template <int ID, int N>
+struct GroupBarrier {
+  __device__ static __forceinline__ void sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
+  }
+};
+
 template <int NL>
 struct SelectState {
   uint64_t prefix[NL];
@@ -24,20 +36,20 @@ struct SelectState {
 // For each list l < NL (keys[l*stride .. l*stride + n[l])), compute T[l] such
 // that exactly kk[l] keys are >= T[l] (keys unique, kk[l] >= 1).  A list
 // with n[l] <= kk[l] gets T[l] = 0 (keep all).  n, kk and T live in shared
-// memory; every thread of the CTA must call this; on return every thread
-// may read T.
-template <int NT, int NL>
+// memory.  Every one of the NT threads synchronised by Bar must call this
+// with its index tid in [0, NT); on return all of them may read T.
+template <int NT, int NL, class Bar = CtaBarrier>
 __device__ void cta_select_thresholds(const uint64_t* keys, int stride,
                                       const int* n, const int* kk, uint64_t* T,
-                                      SelectState<NL>* st) {
+                                      SelectState<NL>* st, int tid) {
   static_assert(NL * 32 <= NT, "one warp per list for the bucket scan");
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid < NL) {
     st->prefix[tid] = 0;
     st->need[tid] = (uint32_t)kk[tid];
     st->done[tid] = n[tid] <= kk[tid];
   }
-  __syncthreads();
+  Bar::sync();
 #pragma unroll 1
   for (int shift = 56; shift >= 0; shift -= 8) {
     bool all_done = true;
@@ -46,7 +58,7 @@ __device__ void cta_select_thresholds(const uint64_t* keys, int stride,
     if (all_done) break;  // uniform: every thread reads the same state
     const uint64_t hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
     for (int b = tid; b < NL * 256; b += NT) st->hist[b] = 0;
-    __syncthreads();
+    Bar::sync();
 #pragma unroll
     for (int l = 0; l < NL; ++l) {
       if (st->done[l]) continue;
@@ -54,12 +66,12 @@ __device__ void cta_select_thresholds(const uint64_t* keys, int stride,
       const uint64_t pf = st->prefix[l];
       const int nl = n[l];
       for (int e = tid; e < nl; e += NT) {
-        uint64_t key = kl[e];
+        const uint64_t key = kl[e];
         if ((key & hmask) == pf)
           atomicAdd(&st->hist[l * 256 + ((uint32_t)(key >> shift) & 255u)], 1u);
       }
     }
-    __syncthreads();
+    Bar::sync();
     if (warp < NL && !st->done[warp]) {
       const uint32_t* h = st->hist + warp * 256;
       uint32_t c[8], sum = 0;
@@ -92,10 +104,10 @@ __device__ void cta_select_thresholds(const uint64_t* keys, int stride,
         }
       }
     }
-    __syncthreads();
+    Bar::sync();
   }
   if (tid < NL) T[tid] = (n[tid] <= kk[tid]) ? 0ull : st->prefix[tid];
-  __syncthreads();
+  Bar::sync();
 }
 
 }  // namespace ca

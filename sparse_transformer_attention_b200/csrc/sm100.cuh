@@ -87,6 +87,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
+// Bulk (non-tensor) copy of `bytes` contiguous bytes from global to shared
+// memory, completing on `bar`.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src,
+                                          uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile(

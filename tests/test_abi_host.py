@@ -108,8 +108,9 @@ def test_invalid_arguments_rejected_before_launch(lib, call, over, code):
     assert call(lib, **over) == code
 
 
-def test_prefill_k_limit(lib):
+def test_k_limits(lib):
     assert _prefill(lib, k=65, C_max=1 + 64 + 65) == binding.CA_ERR_UNSUPPORTED
+    assert _decode(lib, k=1025, C_max=1000) == binding.CA_ERR_UNSUPPORTED
 
 
 def test_small_sequence_needs_only_n_slots(lib):

@@ -63,9 +63,9 @@ def test_noalloc_matches_workspace_entry_point(dtype, tol):
 
 def test_noalloc_rejects_problems_beyond_its_buffer():
     lib = binding.load()
-    # 64 q-heads x 2 chunks x k=4096 candidate keys x 8 bytes = 4 MiB, plus
-    # the status area: one byte past the built-in buffer.
-    w = workloads.get("decode_131k").scaled(n=9000, Hq=64, Hkv=8, k=4096)
+    # 64 q-heads x 8 chunks x k=1024 candidate keys x 8 bytes = 4 MiB, plus
+    # the status area: past the built-in buffer.
+    w = workloads.get("decode_131k").scaled(n=9000, Hq=64, Hkv=8, k=1024)
     assert ca.condensate_attn_workspace_size(
         True, torch.bfloat16, w.B, w.n, w.Hq, w.Hkv, w.d, w.W, w.k) > 4 << 20
     q = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
