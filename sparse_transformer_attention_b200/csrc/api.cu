@@ -142,7 +142,9 @@ ca_status condensate_attn_prefill(const void* Q, const void* K, const void* V,
   a.W_i = W_i; a.O = O; a.o_bf16 = o_dtype == CA_BF16;
   a.idx = idx; a.idx_count = idx_count; a.C_max = C_max;
   a.status = (uint32_t*)workspace;
+  a.ovf_count = (uint32_t*)workspace + 4;  // inside the cleared status area
   a.topk = (uint64_t*)((char*)workspace + ca::kStatusBytes);
+  a.ovf_rows = (uint32_t*)((char*)a.topk + ca::prefill_topk_bytes(B, n, Hq, k));
   cudaError_t e = ca::prefill_launch(a, dtype == CA_BF16, d, s);
   if (e == cudaErrorNotSupported) return CA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;

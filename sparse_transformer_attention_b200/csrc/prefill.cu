@@ -23,7 +23,9 @@
 #include "prefill.cuh"
 #include "profile.cuh"
 #include "row_topk.cuh"
+#include "select.cuh"
 #include "sm100.cuh"
+#include "warp_sort.cuh"
 
 namespace ca {
 
@@ -55,21 +57,37 @@ __device__ void tile_rows(const PrefillArgs& a, int b, int i0, int* s_hi,
 }
 
 // ============================================================ tcgen05 kernel
+// Two passes over the row tile's key tiles (the tensor pipe has room for
+// them; the selector is what costs):
+//   pass 1: every selector thread keeps, for its query row, the maximum over
+//           each of 32 column positions of its 32-column chunk of every key
+//           tile (128 slots per row over the four chunk groups).  The k-th
+//           largest slot maximum L is a lower bound of the row's k-th best
+//           score: the top k slots are k distinct candidates, all >= L.
+//   pass 2: recompute the scores and append every candidate with score >= L
+//           to the row's buffer (about 1.1-1.4 k entries on random data).
+// The exact Top-k is then taken from the buffer with a small heap.  A row
+// whose buffer would overflow is listed for an exact CUDA-core fallback.
+constexpr int kSelWarps = 16;                       // 4 chunk groups x 4 quarters
+constexpr int kTcThreads = 64 + 32 * kSelWarps;     // + TMA warp + MMA warp
+constexpr int kMinCap = 64;                         // the slot table needs 64 KiB
+using SelBar = GroupBarrier<1, 32 * kSelWarps>;
+
 template <int D>
 struct TcLayout {
   static constexpr int BM = 128, BN = 128;
   static constexpr int KB = D / 64;                   // 128-byte column blocks
   static constexpr int NS = (D == 64) ? 4 : 2;        // K stages
-  static constexpr int S = (D == 64) ? 64 : 32;       // staging slots per row
   static constexpr uint32_t kQBytes = BM * D * 2;
   static constexpr uint32_t kKBytes = BN * D * 2;
   static constexpr uint32_t kBlockBytes = 128 * 128;  // 128 rows x 128 bytes
   static constexpr size_t q_off = 0;
   static constexpr size_t k_off = q_off + kQBytes;
-  static constexpr size_t heap_off = k_off + (size_t)NS * kKBytes;
-  __host__ __device__ static size_t stage_off(int k) { return heap_off + (size_t)k * kTileRows * 8; }
-  __host__ __device__ static size_t bar_off(int k) { return stage_off(k) + (size_t)S * kTileRows * 8; }
-  __host__ __device__ static size_t bytes(int k) { return bar_off(k) + 256 + 1024; }  // + align
+  static constexpr size_t buf_off = k_off + (size_t)NS * kKBytes;
+  // row buffers [cap][128] keys; + 1 KiB for the manual 1024-byte alignment
+  __host__ __device__ static size_t bytes(int cap) {
+    return buf_off + (size_t)cap * kTileRows * 8 + 1024;
+  }
 };
 
 struct TcShared {
@@ -78,6 +96,9 @@ struct TcShared {
   int abort;
   int maxhi;
   int hi[kTileRows];
+  float L[kTileRows];
+  int cnt[kTileRows];
+  int ovf[kTileRows];
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
@@ -96,10 +117,36 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Min-heap of k keys for row r, stored at h[e * 128 + r]; replace the root
+// by `key` (> root) and sift down.
+__device__ __forceinline__ uint64_t heap_replace(uint64_t* h, int k, int r,
+                                                 uint64_t key) {
+  int p = 0;
+#pragma unroll 1
+  while (true) {
+    int c = 2 * p + 1;
+    if (c >= k) break;
+    uint64_t cv = h[c * kTileRows + r];
+    if (c + 1 < k) {
+      const uint64_t c2 = h[(c + 1) * kTileRows + r];
+      if (c2 < cv) {
+        cv = c2;
+        c = c + 1;
+      }
+    }
+    if (cv >= key) break;
+    h[p * kTileRows + r] = cv;
+    p = c;
+  }
+  h[p * kTileRows + r] = key;
+  return h[r];
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmK, PrefillArgs a) {
+                      const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
+                      int cap) {
   using Lay = TcLayout<D>;
   constexpr int BN = Lay::BN, NS = Lay::NS, KB = Lay::KB;
   extern __shared__ unsigned char smem_raw[];
@@ -107,16 +154,22 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = smem + Lay::q_off;
   unsigned char* sK = smem + Lay::k_off;
-  uint64_t* heap = reinterpret_cast<uint64_t*>(smem + Lay::heap_off);
-  uint2* stage = reinterpret_cast<uint2*>(smem + Lay::stage_off(a.k));
+  uint64_t* rbuf = reinterpret_cast<uint64_t*>(smem + Lay::buf_off);
+  float* table = reinterpret_cast<float*>(smem + Lay::buf_off);  // pass-1 slots
+  uint64_t* heap = reinterpret_cast<uint64_t*>(sK);  // K ring, free at the end
   __shared__ TcShared sh;
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (a.Hq / a.Hkv);
   const int i0 = qt * Lay::BM;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k = a.k;
 
   tile_rows(a, b, i0, sh.hi, &sh.maxhi);
+  if (tid < kTileRows) {
+    sh.cnt[tid] = 0;
+    sh.ovf[tid] = 0;
+  }
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       sm100::mbar_init(&sh.kfull[s], 1);
@@ -125,7 +178,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sm100::mbar_init(&sh.qfull, 1);
     for (int t = 0; t < 2; ++t) {
       sm100::mbar_init(&sh.tfull[t], 1);
-      sm100::mbar_init(&sh.tempty[t], 4);
+      sm100::mbar_init(&sh.tempty[t], kSelWarps);
     }
     sh.abort = 0;
     sm100::fence_barrier_init();
@@ -140,10 +193,11 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t tmem = sh.tmem;
   const int maxhi = sh.maxhi;
   const int T = maxhi >= 1 ? maxhi / BN + 1 : 0;  // key tiles with candidates
+  const int TT = 2 * T;                           // two passes
   volatile int* abort_flag = &sh.abort;
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer: key tiles 0..T-1, twice
     if (lane == 0 && T > 0) {
       sm100::prefetch_tmap(&tmQ);
       sm100::prefetch_tmap(&tmK);
@@ -154,8 +208,9 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         sm100::tma_load_2d(sQ + kb * Lay::kBlockBytes, &tmQ, &sh.qfull, kb * 64,
                            qrow);
       int issued = 0;
-      for (int t = 0; t < T; ++t) {
+      for (int t = 0; t < TT; ++t) {
         const int s = t % NS;
+        const int tile = t < T ? t : t - T;
         if (t >= NS &&
             !wait_or_abort(&sh.kempty[s], ((t / NS) & 1) ^ 1, abort_flag,
                            a.status))
@@ -164,7 +219,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         unsigned char* dst = sK + (size_t)s * Lay::kKBytes;
         for (int kb = 0; kb < KB; ++kb)
           sm100::tma_load_2d(dst + kb * Lay::kBlockBytes, &tmK, &sh.kfull[s],
-                             kb * 64, krow + t * BN);
+                             kb * 64, krow + tile * BN);
         issued = t + 1;
       }
       // Let every copy this thread started land before the CTA can exit.
@@ -180,7 +235,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       const uint32_t ak = sm100::smem_u32(sK);
       int done = 0;
       if (wait_or_abort(&sh.qfull, 0, abort_flag, a.status)) {
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; t < TT; ++t) {
           const int s = t % NS, buf = t & 1;
           if (!wait_or_abort(&sh.kfull[s], (t / NS) & 1, abort_flag, a.status))
             break;
@@ -207,42 +262,120 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                          kWaitLimitNs);
     }
   } else {
-    // ---------------- selector warps 2..5: thread = query row
-    const int quarter = warp & 3;
+    // ---------------- selector warps: thread = query row, group = chunk
+    const int sw = warp - 2;               // 0..15
+    const int grp = sw >> 2;               // 32-column chunk of every tile
+    const int quarter = warp & 3;          // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
-    const int i = i0 + r;
     const int hi = sh.hi[r];
-    RowTopk sel;
-    sel.init(heap, stage, r, a.k, Lay::S);
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    for (int t = 0; t < T; ++t) {
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + grp * 32;
+
+    // ---- pass 1: slot maxima
+    float colmax[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) colmax[x] = -INFINITY;
+    int t = 0;
+    for (; t < T; ++t) {
       const int buf = t & 1;
-      // warp-uniform: tcgen05.ld below needs every lane of the warp
       if (!__all_sync(0xFFFFFFFFu, wait_or_abort(&sh.tfull[buf], (t >> 1) & 1,
                                                  abort_flag, a.status)))
         break;
       sm100::tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t raw[32];
-        sm100::tmem_ld_32x32b_x32(tl + buf * BN + c * 32, raw);
-        sm100::tmem_wait_ld();
-        if (c == BN / 32 - 1) {
-          sm100::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
-        }
-        const int j0 = t * BN + c * 32;
-        const bool interior = (j0 >= 1) && (j0 + 31 <= hi);
-        if (__all_sync(0xFFFFFFFFu, interior))
-          sel.offer<false>(raw, j0, 1, hi);
-        else
-          sel.offer<true>(raw, j0, 1, hi);
+      uint32_t raw[32];
+      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
+      sm100::tmem_wait_ld();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
+      const int j0 = t * BN + grp * 32;
+      if (__all_sync(0xFFFFFFFFu, j0 >= 1 && j0 + 31 <= hi)) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (j0 + x >= 1 && j0 + x <= hi)
+            colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
       }
     }
-    sel.drain();
-    if (i < a.n && a.k > 0)
-      sel.store(a.topk + ((size_t)(b * a.Hq + h) * a.n + i) * a.k);
+    // ---- bound: k-th largest of the row's 128 slot maxima.  The table
+    // row is stored with its 16-byte pieces XOR-swizzled by the row index so
+    // that 32 rows written (or one row read) at once spread over the banks.
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int piece = (grp * 8 + c) ^ (r & 31);
+      *reinterpret_cast<float4*>(table + r * 128 + piece * 4) =
+          make_float4(colmax[4 * c], colmax[4 * c + 1], colmax[4 * c + 2],
+                      colmax[4 * c + 3]);
+    }
+    SelBar::sync();
+    for (int rr = 0; rr < 8; ++rr) {
+      const int row = sw * 8 + rr;
+      const int piece = lane ^ (row & 31);
+      const float4 v = *reinterpret_cast<const float4*>(table + row * 128 +
+                                                         piece * 4);
+      uint32_t key[4] = {ord_f32(v.x), ord_f32(v.y), ord_f32(v.z),
+                         ord_f32(v.w)};
+      warp_bitonic<4>(key, lane);  // ascending over 128 slots
+      const int e = 128 - k;       // the k-th largest
+      const uint32_t kk = __shfl_sync(0xFFFFFFFFu, key[e >> 5], e & 31);
+      if (lane == 0)
+        sh.L[row] = (kk <= ord_f32(-INFINITY)) ? -INFINITY : unord_f32(kk);
+    }
+    SelBar::sync();
+    const float Lr = sh.L[r];
+    // ---- pass 2: append every candidate >= L
+    for (; t < TT; ++t) {
+      const int buf = t & 1;
+      if (!__all_sync(0xFFFFFFFFu, wait_or_abort(&sh.tfull[buf], (t >> 1) & 1,
+                                                 abort_flag, a.status)))
+        break;
+      sm100::tc_fence_after();
+      uint32_t raw[32];
+      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
+      sm100::tmem_wait_ld();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
+      const int j0 = (t - T) * BN + grp * 32;
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        const bool p = j0 + x >= 1 && j0 + x <= hi &&
+                       __uint_as_float(raw[x]) >= Lr;
+        if (__any_sync(0xFFFFFFFFu, p) && p) {
+          const int pos = atomicAdd(&sh.cnt[r], 1);
+          if (pos < cap)
+            rbuf[(size_t)pos * kTileRows + r] =
+                make_key(__uint_as_float(raw[x]), (uint32_t)(j0 + x));
+          else
+            sh.ovf[r] = 1;
+        }
+      }
+    }
+    SelBar::sync();
+    // ---- exact Top-k of the row's buffer (one thread per row)
+    if (grp == 0) {
+      const int i = i0 + r;
+      if (i < a.n && k > 0) {
+        const size_t grow = (size_t)(b * a.Hq + h) * a.n + i;
+        uint64_t* out = a.topk + grow * k;
+        if (sh.ovf[r]) {
+          // listed for the exact fallback pass; it writes this row
+          const uint32_t pos = atomicAdd(a.ovf_count, 1u);
+          a.ovf_rows[pos] = (uint32_t)grow;
+        } else {
+          for (int e = 0; e < k; ++e) heap[e * kTileRows + r] = 0ull;
+          uint64_t root = 0ull;
+          const int n = sh.cnt[r];
+          for (int e = 0; e < n; ++e) {
+            const uint64_t key = rbuf[(size_t)e * kTileRows + r];
+            if (key > root) root = heap_replace(heap, k, r, key);
+          }
+          for (int e = 0; e < k; ++e) out[e] = heap[e * kTileRows + r];
+        }
+      }
+    }
   }
   __syncwarp();  // reconverge single-lane roles before the CTA barrier
   sm100::tc_fence_before();
@@ -250,6 +383,74 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   if (warp == 1) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, 256);
+  }
+}
+
+// Exact fallback for rows whose candidate buffer overflowed: one CTA per
+// listed row scores every candidate on CUDA cores (fp32 FMA of the bf16 or
+// fp32 inputs) and keeps the best k keys with the CTA radix select.
+constexpr int kFbThreads = 256;
+constexpr int kFbChunk = 2048;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kFbThreads)
+prefill_overflow_rows(PrefillArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int k = a.k;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);      // [k + chunk]
+  float* q = reinterpret_cast<float*>(keys + k + kFbChunk);  // [D]
+  __shared__ int s_n, s_kk, s_w;
+  __shared__ uint64_t s_T;
+  __shared__ SelectState<1> st;
+  const uint32_t nrows = *a.ovf_count;
+  for (uint32_t it = blockIdx.x; it < nrows; it += gridDim.x) {
+    const uint32_t grow = a.ovf_rows[it];
+    const int i = (int)(grow % (uint32_t)a.n);
+    const uint32_t bh = grow / (uint32_t)a.n;
+    const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
+    const int g = h / (a.Hq / a.Hkv);
+    const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n, a.status,
+                             false);
+    const int hi = i - w;
+    const T* Qr = reinterpret_cast<const T*>(a.Q) + (size_t)grow * D;
+    const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * a.n * D;
+    for (int e = threadIdx.x; e < D; e += kFbThreads) q[e] = Elem<T>::load1(Qr + e);
+    if (threadIdx.x == 0) s_n = 0;
+    __syncthreads();
+    for (int c0 = 1; c0 <= hi; c0 += kFbChunk) {
+      for (int jj = threadIdx.x; jj < kFbChunk && c0 + jj <= hi; jj += kFbThreads) {
+        const int j = c0 + jj;
+        const T* kr = Kg + (size_t)j * D;
+        float acc = 0.f;
+        for (int e = 0; e < D; ++e) acc = fmaf(q[e], Elem<T>::load1(kr + e), acc);
+        keys[s_n + jj] = make_key(acc, (uint32_t)j);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        s_n += (hi - c0 + 1 < kFbChunk) ? (hi - c0 + 1) : kFbChunk;
+        s_kk = k;
+      }
+      __syncthreads();
+      cta_select_thresholds<kFbThreads, 1>(keys, 0, &s_n, &s_kk, &s_T, &st,
+                                           threadIdx.x);
+      if (s_n > k) {
+        // keep the keys >= T, packed to the front
+        if (threadIdx.x == 0) s_w = 0;
+        __syncthreads();
+        uint64_t mine[(kPrefillMaxK + kFbChunk) / kFbThreads + 1];
+        int cntm = 0;
+        for (int e = threadIdx.x; e < s_n; e += kFbThreads) mine[cntm++] = keys[e];
+        __syncthreads();
+        for (int c = 0; c < cntm; ++c)
+          if (mine[c] >= s_T) keys[atomicAdd(&s_w, 1)] = mine[c];
+        __syncthreads();
+        if (threadIdx.x == 0) s_n = k;
+        __syncthreads();
+      }
+    }
+    uint64_t* out = a.topk + (size_t)grow * k;
+    for (int e = threadIdx.x; e < k; e += kFbThreads) out[e] = e < s_n ? keys[e] : 0ull;
+    __syncthreads();
   }
 }
 
@@ -531,14 +732,29 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, a.Q, (uint64_t)a.B * a.Hq * a.n, D)) return cudaErrorInvalidValue;
   if (!make_tmap(&tk, a.K, (uint64_t)a.B * a.Hkv * a.n, D)) return cudaErrorInvalidValue;
-  const size_t smem = Lay::bytes(a.k);
+  // row buffer: 3k candidates (the pass-1 bound leaves about 1.1-1.4 k),
+  // at least kMinCap slots, at most what fits next to Q and the K ring
+  const size_t budget = 227 * 1024 - sizeof(TcShared);
+  const int cap_max = (int)((budget - Lay::bytes(0)) / (kTileRows * 8));
+  int cap = 3 * a.k;
+  if (cap < kMinCap) cap = kMinCap;
+  if (cap > cap_max) cap = cap_max;
+  if (cap < a.k || cap < kMinCap) return cudaErrorNotSupported;
+  const size_t smem = Lay::bytes(cap);
   auto kern = prefill_score_topk_tc<D>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_tc");
-  kern<<<grid, 192, smem, s>>>(tq, tk, a);
+  kern<<<grid, kTcThreads, smem, s>>>(tq, tk, a, cap);
+  prof_after(s);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // rows whose buffer overflowed (none on typical inputs): exact fallback
+  const size_t fb_smem = (size_t)(a.k + kFbChunk) * 8 + D * 4;
+  prof_before(s, "prefill_overflow_rows");
+  prefill_overflow_rows<__nv_bfloat16, D><<<148, kFbThreads, fb_smem, s>>>(a);
   prof_after(s);
   return cudaGetLastError();
 }
@@ -578,9 +794,15 @@ cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-size_t prefill_workspace(bool, int B, int n, int Hq, int, int, int k) {
+size_t prefill_topk_bytes(int B, int n, int Hq, int k) {
   size_t bytes = (size_t)B * Hq * n * (size_t)(k > 0 ? k : 1) * 8;
   return (bytes + 255) / 256 * 256;
+}
+
+size_t prefill_workspace(bool, int B, int n, int Hq, int, int, int k) {
+  // per-row Top-k keys, then the list of rows for the exact fallback
+  return prefill_topk_bytes(B, n, Hq, k) +
+         ((size_t)B * Hq * n * 4 + 255) / 256 * 256;
 }
 
 cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,

@@ -23,8 +23,12 @@ struct PrefillArgs {
   int C_max;
   uint32_t* status;  // device status word (workspace)
   uint64_t* topk;    // [B*Hq*n, k] selected keys per row (workspace)
+  uint32_t* ovf_count;  // rows listed for the exact fallback (status area)
+  uint32_t* ovf_rows;   // [B*Hq*n] their row indices (workspace)
 };
 
+// Bytes of the per-row Top-k key area at the start of the workspace body.
+size_t prefill_topk_bytes(int B, int n, int Hq, int k);
 // Workspace bytes beyond the status area.
 size_t prefill_workspace(bool bf16, int B, int n, int Hq, int Hkv, int d,
                          int k);

@@ -78,3 +78,15 @@ def test_prefill_adaptive_32k_sampled():
     w = workloads.get("prefill_adaptive_32k")
     x = workloads.generate(w)
     print(check_prefill(w, x, W_i=x["W_i"], sel=_sample_rows(w, 600, 1)))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_equal_keys_take_the_fallback(d):
+    """All keys equal: every candidate ties at the pass-1 bound, so rows with
+    more candidates than the row buffer holds go through the exact fallback;
+    ties go to the lowest indices."""
+    w = workloads.get("prefill_gpt2s_8k").scaled(d=d, n=700, B=1, Hq=2, Hkv=2,
+                                                 needles=0)
+    x = workloads.generate(w)
+    x["K"][:] = x["K"][:, :, :1, :]
+    print(check_prefill(w, x))
