@@ -325,6 +325,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     }
     SelBar::sync();
     const float Lr = sh.L[r];
+    bool ovf_local = false;
     // ---- pass 2: append every candidate >= L
     for (; t < TT; ++t) {
       const int buf = t & 1;
@@ -339,20 +340,36 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
       const int j0 = (t - T) * BN + grp * 32;
+      // A score can only qualify if it reaches L; one warp vote per column
+      // keeps the (rare) append off the common path.
+      auto append = [&](uint32_t bits, int j) {
+        const int pos = atomicAdd(&sh.cnt[r], 1);
+        if (pos < cap)
+          rbuf[(size_t)pos * kTileRows + r] = make_key(__uint_as_float(bits),
+                                                       (uint32_t)j);
+        else
+          ovf_local = true;
+      };
+      if (__all_sync(0xFFFFFFFFu, j0 >= 1 && j0 + 31 <= hi)) {
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const bool p = j0 + x >= 1 && j0 + x <= hi &&
-                       __uint_as_float(raw[x]) >= Lr;
-        if (__any_sync(0xFFFFFFFFu, p) && p) {
-          const int pos = atomicAdd(&sh.cnt[r], 1);
-          if (pos < cap)
-            rbuf[(size_t)pos * kTileRows + r] =
-                make_key(__uint_as_float(raw[x]), (uint32_t)(j0 + x));
-          else
-            sh.ovf[r] = 1;
+        for (int x = 0; x < 32; ++x) {
+          const bool p = __uint_as_float(raw[x]) >= Lr;
+          if (__any_sync(0xFFFFFFFFu, p)) {
+            if (p) append(raw[x], j0 + x);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const bool p = j0 + x >= 1 && j0 + x <= hi &&
+                         __uint_as_float(raw[x]) >= Lr;
+          if (__any_sync(0xFFFFFFFFu, p)) {
+            if (p) append(raw[x], j0 + x);
+          }
         }
       }
     }
+    if (ovf_local) sh.ovf[r] = 1;
     SelBar::sync();
     // ---- exact Top-k of the row's buffer (one thread per row)
     if (grp == 0) {
