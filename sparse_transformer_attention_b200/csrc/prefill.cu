@@ -65,13 +65,25 @@ __device__ void tile_rows(const PrefillArgs& a, int b, int i0, int* s_hi,
 //           largest slot maximum L is a lower bound of the row's k-th best
 //           score: the top k slots are k distinct candidates, all >= L.
 //   pass 2: recompute the scores and append every candidate with score >= L
-//           to the row's buffer (about 1.1-1.4 k entries on random data).
-// The exact Top-k is then taken from the buffer with a small heap.  A row
-// whose buffer would overflow is listed for an exact CUDA-core fallback.
+//           to the thread's own segment (about 1.1-1.4 k entries per row on
+//           random data), with predicated stores and no atomics.
+// The exact Top-k is then found per row by one warp (bisection on the key
+// bits over the row's four segments).  A row whose segment would overflow is
+// listed for an exact CUDA-core fallback.
 constexpr int kSelWarps = 16;                       // 4 chunk groups x 4 quarters
-constexpr int kTcThreads = 64 + 32 * kSelWarps;     // + TMA warp + MMA warp
-constexpr int kMinCap = 64;                         // the slot table needs 64 KiB
-using SelBar = GroupBarrier<1, 32 * kSelWarps>;
+constexpr int kSelThreads = 32 * kSelWarps;         // (row, chunk group) pairs
+constexpr int kTcThreads = 64 + kSelThreads;        // + TMA warp + MMA warp
+constexpr int kTmemBufs = 4;                        // 128-column accumulators
+constexpr int kMinSeg = 16;                         // smallest segment (entries)
+constexpr int kPoolCols = 16;                       // spare segments per CTA
+constexpr int kSegCols = kSelThreads + kPoolCols;   // segment columns
+constexpr int kScoreStride = (kSegCols + 1) * 4;    // bytes between positions
+constexpr int kCodeStride = (kSegCols + 2) * 2;     // (odd word strides: the
+                                                    //  entries of one column
+                                                    //  spread over the banks)
+constexpr uint32_t kMaskedScore = 0x7FC00000u;      // NaN: never >= L, ignored
+                                                    // by fmaxf
+using SelBar = GroupBarrier<1, kSelThreads>;
 
 template <int D>
 struct TcLayout {
@@ -83,22 +95,30 @@ struct TcLayout {
   static constexpr uint32_t kBlockBytes = 128 * 128;  // 128 rows x 128 bytes
   static constexpr size_t q_off = 0;
   static constexpr size_t k_off = q_off + kQBytes;
-  static constexpr size_t buf_off = k_off + (size_t)NS * kKBytes;
-  // row buffers [cap][128] keys; + 1 KiB for the manual 1024-byte alignment
-  __host__ __device__ static size_t bytes(int cap) {
-    return buf_off + (size_t)cap * kTileRows * 8 + 1024;
+  static constexpr size_t seg_off = k_off + (size_t)NS * kKBytes;
+  // Segments: P positions of scores (u32) then of codes (u16); the pass-1
+  // slot table (128 rows x 128 fp32) uses the same bytes first.
+  __host__ __device__ static size_t code_off(int P) {
+    return seg_off + ((size_t)P * kScoreStride + 15) / 16 * 16;
+  }
+  __host__ __device__ static size_t bytes(int P) {
+    size_t seg = code_off(P) - seg_off + (size_t)P * kCodeStride;
+    if (seg < (size_t)kTileRows * 128 * 4) seg = (size_t)kTileRows * 128 * 4;
+    return seg_off + seg + 1024;  // + the manual 1024-byte alignment
   }
 };
 
 struct TcShared {
-  uint64_t kfull[4], kempty[4], qfull, tfull[2], tempty[2];
+  uint64_t kfull[4], kempty[4], qfull, tfull[kTmemBufs], tempty[kTmemBufs];
   uint32_t tmem;
   int abort;
   int maxhi;
   int hi[kTileRows];
   float L[kTileRows];
-  int cnt[kTileRows];
-  int ovf[kTileRows];
+  short cnt[kSelThreads];   // entries in the thread's own segment, -1: overflow
+  short xcnt[kSelThreads];  // entries in its spare segment
+  signed char xcol[kSelThreads];  // spare segment index, -1: none
+  int pool;                 // spare segments handed out
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
@@ -117,36 +137,243 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   }
 }
 
-// Min-heap of k keys for row r, stored at h[e * 128 + r]; replace the root
-// by `key` (> root) and sift down.
-__device__ __forceinline__ uint64_t heap_replace(uint64_t* h, int k, int r,
-                                                 uint64_t key) {
-  int p = 0;
+// Append (score, code) at the segment cursor when score >= L; predicated
+// stores, so a warp never branches on the comparison.
+__device__ __forceinline__ void seg_append(uint32_t& as, uint32_t& ac,
+                                           uint32_t bits, float L,
+                                           uint32_t code) {
+  asm volatile(
+      "{ .reg .pred p; .reg .b16 c;\n\t"
+      "setp.ge.f32 p, %2, %3;\n\t"
+      "cvt.u16.u32 c, %5;\n\t"
+      "@p st.shared.b32 [%0], %4;\n\t"
+      "@p st.shared.b16 [%1], c;\n\t"
+      "@p add.u32 %0, %0, %6;\n\t"
+      "@p add.u32 %1, %1, %7; }"
+      : "+r"(as), "+r"(ac)
+      : "f"(__uint_as_float(bits)), "f"(L), "r"(bits), "r"(code),
+        "n"(kScoreStride), "n"(kCodeStride)
+      : "memory");
+}
+
+// Append the 32 scores of one key tile chunk.  Cursors are checked every 8
+// columns: a cursor past `*_max` (8 positions before the end) is clamped
+// and `full` is set, and the caller redoes the tile elsewhere.
+__device__ __forceinline__ void append_tile(const uint32_t (&raw)[32],
+                                            uint32_t& as, uint32_t& ac,
+                                            float L, uint32_t cbase,
+                                            uint32_t as_max, uint32_t ac_max,
+                                            bool& full) {
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    seg_append(as, ac, raw[x], L, cbase + x);
+    if ((x & 7) == 7) {
+      full |= as > as_max;
+      as = min(as, as_max);
+      ac = min(ac, ac_max);
+    }
+  }
+}
+
+// Segments of one row: slot g < 4 is chunk group g's own segment (column
+// g * 128 + row), slot 4 + g its spare one (column 512 + spare index, empty
+// when there is none).  Entry f lives in the last slot s with start[s] <= f
+// (empty slots share the start of the next one).
+struct RowSegs {
+  int n;           // entries of the row
+  int row;         // row within the tile
+  int start[8];    // prefix of the slot counts
+  int xcolm[4];    // spare segment column of each group
+  bool bad;        // a segment overflowed
+};
+
+__device__ __forceinline__ void row_segs(const TcShared& sh, int row,
+                                         RowSegs& q) {
+  q.row = row;
+  q.n = 0;
+  q.bad = false;
+#pragma unroll
+  for (int gq = 0; gq < 4; ++gq) {
+    const int c = sh.cnt[gq * kTileRows + row];
+    q.bad |= c < 0;
+    q.start[gq] = q.n;
+    q.n += c < 0 ? 0 : c;
+  }
+#pragma unroll
+  for (int gq = 0; gq < 4; ++gq) {
+    const int x = sh.xcol[gq * kTileRows + row];
+    q.start[4 + gq] = q.n;
+    q.xcolm[gq] = kSelThreads + (x < 0 ? 0 : x);
+    if (x >= 0) q.n += sh.xcnt[gq * kTileRows + row];
+  }
+}
+
+__device__ __forceinline__ void seg_locate(const RowSegs& rs, int f, int& col,
+                                           int& grp, int& e) {
+  int s = 0;
+#pragma unroll
+  for (int q = 1; q < 8; ++q) s += f >= rs.start[q];
+  int st = rs.start[0];
+#pragma unroll
+  for (int q = 1; q < 8; ++q)
+    if (q == s) st = rs.start[q];
+  int xcol = rs.xcolm[0];
+#pragma unroll
+  for (int q = 1; q < 4; ++q)
+    if (q == (s & 3)) xcol = rs.xcolm[q];
+  grp = s & 3;
+  col = s < 4 ? grp * kTileRows + rs.row : xcol;
+  e = f - st;
+}
+
+__device__ __forceinline__ uint32_t seg_hi(const unsigned char* seg, int col,
+                                           int e) {
+  const uint32_t bits = *reinterpret_cast<const uint32_t*>(
+      seg + (size_t)e * kScoreStride + col * 4);
+  return ord_f32(__uint_as_float(bits));
+}
+
+__device__ __forceinline__ uint32_t seg_lo(const unsigned char* codes,
+                                           int col, int grp, int e) {
+  const uint32_t code = *reinterpret_cast<const uint16_t*>(
+      codes + (size_t)e * kCodeStride + col * 2);
+  const uint32_t j = (code >> 5) * 128 + grp * 32 + (code & 31);
+  return 0xFFFFFFFFu - j;
+}
+
+// Sum over the four lanes of a row group.
+__device__ __forceinline__ int quad_sum(int v) {
+  v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+  return v + __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+}
+
+// Exact Top-k of the rows of one warp, four lanes per row (lane & 3 = part;
+// entry f of the row is held by part f & 3).  `sel` rows take the k largest
+// keys (ord(score), ~j) of their n entries, found by bisection on the score
+// bits (and on the index bits only when equal scores straddle the cut);
+// `all` rows (n <= k) take every entry.  The selected keys go to out[0..) in
+// any order, padded with empty keys.  Missing entries hold 0, below every
+// probe.
+template <int NE>
+__device__ __forceinline__ void quad_select(const unsigned char* seg,
+                                            const unsigned char* codes,
+                                            const RowSegs& rs, bool live,
+                                            uint32_t lob, int k, uint64_t* out,
+                                            int part) {
+  uint32_t hv[NE];
+#pragma unroll
+  for (int t = 0; t < NE; ++t) {
+    const int f = part + 4 * t;
+    hv[t] = 0u;
+    if (live && f < rs.n) {
+      int col, grp, e;
+      seg_locate(rs, f, col, grp, e);
+      hv[t] = seg_hi(seg, col, e);
+    }
+  }
+  const bool sel = live && rs.n > k;
+  // bisection start: the common high bits of the bound and the row maximum
+  uint32_t mx = 0u;
+#pragma unroll
+  for (int t = 0; t < NE; ++t) mx = max(mx, hv[t]);
+  mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+  mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+  const uint32_t diff = lob ^ mx;
+  const int nb = sel ? (diff ? 32 - __clz(diff) : 0) : 0;
+  uint32_t tau = nb == 32 ? 0u : (lob >> nb) << nb;
+  bool done = nb == 0, exact = false;
+  const int bmax = __reduce_max_sync(0xFFFFFFFFu, nb);
 #pragma unroll 1
-  while (true) {
-    int c = 2 * p + 1;
-    if (c >= k) break;
-    uint64_t cv = h[c * kTileRows + r];
-    if (c + 1 < k) {
-      const uint64_t c2 = h[(c + 1) * kTileRows + r];
-      if (c2 < cv) {
-        cv = c2;
-        c = c + 1;
+  for (int b = bmax - 1; b >= 0; --b) {
+    if (__all_sync(0xFFFFFFFFu, done)) break;
+    const uint32_t c = tau | (1u << b);
+    int m = 0;
+#pragma unroll
+    for (int t = 0; t < NE; ++t) m += hv[t] >= c;
+    m = quad_sum(m);
+    const bool up = !done && b < nb && m >= k;
+    tau = up ? c : tau;
+    const bool fin = up && m == k;
+    done |= fin;
+    exact |= fin;
+  }
+  uint32_t th_hi = sel ? tau : 0u, th_lo = 0u;
+  // equal scores straddling the cut: the lower positions win
+  int gt = 0, ge = 0;
+#pragma unroll
+  for (int t = 0; t < NE; ++t) {
+    gt += hv[t] > th_hi;
+    ge += hv[t] >= th_hi;
+  }
+  gt = quad_sum(gt);
+  ge = quad_sum(ge);
+  const int need = (sel && !exact && ge > k) ? k - gt : 0;
+  if (__any_sync(0xFFFFFFFFu, need > 0)) {
+    uint32_t lo[NE];
+#pragma unroll
+    for (int t = 0; t < NE; ++t) {
+      const int f = part + 4 * t;
+      lo[t] = 0u;
+      if (need > 0 && f < rs.n && hv[t] == th_hi) {
+        int col, grp, e;
+        seg_locate(rs, f, col, grp, e);
+        lo[t] = seg_lo(codes, col, grp, e);
       }
     }
-    if (cv >= key) break;
-    h[p * kTileRows + r] = cv;
-    p = c;
+#pragma unroll 1
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t c = th_lo | (1u << b);
+      int m = 0;
+#pragma unroll
+      for (int t = 0; t < NE; ++t) m += hv[t] == th_hi && lo[t] >= c;
+      m = quad_sum(m);
+      th_lo = (need > 0 && m >= need) ? c : th_lo;
+    }
   }
-  h[p * kTileRows + r] = key;
-  return h[r];
+  // write the selected keys: exclusive prefix over the four parts
+  int cnt = 0;
+#pragma unroll
+  for (int t = 0; t < NE; ++t) {
+    const int f = part + 4 * t;
+    if (live && f < rs.n && hv[t] >= th_hi) {
+      bool s = hv[t] > th_hi || th_lo == 0u;
+      if (!s) {
+        int col, grp, e;
+        seg_locate(rs, f, col, grp, e);
+        s = seg_lo(codes, col, grp, e) >= th_lo;
+      }
+      cnt += s;
+    }
+  }
+  const int up1 = __shfl_up_sync(0xFFFFFFFFu, cnt, 1);
+  const int up2 = __shfl_up_sync(0xFFFFFFFFu, cnt, 2);
+  const int up3 = __shfl_up_sync(0xFFFFFFFFu, cnt, 3);
+  const int pre =
+      (part >= 1 ? up1 : 0) + (part >= 2 ? up2 : 0) + (part >= 3 ? up3 : 0);
+  const int total = quad_sum(cnt);
+  if (live) {
+    int pos = pre;
+#pragma unroll
+    for (int t = 0; t < NE; ++t) {
+      const int f = part + 4 * t;
+      if (f < rs.n && hv[t] >= th_hi) {
+        int col, grp, e;
+        seg_locate(rs, f, col, grp, e);
+        const uint32_t lo = seg_lo(codes, col, grp, e);
+        if (hv[t] > th_hi || lo >= th_lo) {
+          out[pos++] = ((uint64_t)hv[t] << 32) | lo;
+        }
+      }
+    }
+    for (int e = total + part; e < k; e += 4) out[e] = 0ull;
+  }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
-                      int cap) {
+                      int P) {
   using Lay = TcLayout<D>;
   constexpr int BN = Lay::BN, NS = Lay::NS, KB = Lay::KB;
   extern __shared__ unsigned char smem_raw[];
@@ -154,9 +381,9 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = smem + Lay::q_off;
   unsigned char* sK = smem + Lay::k_off;
-  uint64_t* rbuf = reinterpret_cast<uint64_t*>(smem + Lay::buf_off);
-  float* table = reinterpret_cast<float*>(smem + Lay::buf_off);  // pass-1 slots
-  uint64_t* heap = reinterpret_cast<uint64_t*>(sK);  // K ring, free at the end
+  unsigned char* seg = smem + Lay::seg_off;     // scores [P][512] (stride 513)
+  unsigned char* codes = smem + Lay::code_off(P);  // codes [P][512] (514)
+  float* table = reinterpret_cast<float*>(seg);  // pass-1 slots, then free
   __shared__ TcShared sh;
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -166,25 +393,22 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   const int k = a.k;
 
   tile_rows(a, b, i0, sh.hi, &sh.maxhi);
-  if (tid < kTileRows) {
-    sh.cnt[tid] = 0;
-    sh.ovf[tid] = 0;
-  }
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       sm100::mbar_init(&sh.kfull[s], 1);
       sm100::mbar_init(&sh.kempty[s], 1);
     }
     sm100::mbar_init(&sh.qfull, 1);
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < kTmemBufs; ++t) {
       sm100::mbar_init(&sh.tfull[t], 1);
       sm100::mbar_init(&sh.tempty[t], kSelWarps);
     }
     sh.abort = 0;
+    sh.pool = 0;
     sm100::fence_barrier_init();
   }
   if (warp == 1) {
-    sm100::tmem_alloc(&sh.tmem, 256);
+    sm100::tmem_alloc(&sh.tmem, kTmemBufs * BN);
     sm100::tmem_relinquish();
   }
   sm100::tc_fence_before();
@@ -208,12 +432,12 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         sm100::tma_load_2d(sQ + kb * Lay::kBlockBytes, &tmQ, &sh.qfull, kb * 64,
                            qrow);
       int issued = 0;
+      int s = 0;
+      uint32_t ph = 0;
       for (int t = 0; t < TT; ++t) {
-        const int s = t % NS;
         const int tile = t < T ? t : t - T;
         if (t >= NS &&
-            !wait_or_abort(&sh.kempty[s], ((t / NS) & 1) ^ 1, abort_flag,
-                           a.status))
+            !wait_or_abort(&sh.kempty[s], ph ^ 1, abort_flag, a.status))
           break;
         sm100::mbar_arrive_expect_tx(&sh.kfull[s], Lay::kKBytes);
         unsigned char* dst = sK + (size_t)s * Lay::kKBytes;
@@ -221,6 +445,10 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
           sm100::tma_load_2d(dst + kb * Lay::kBlockBytes, &tmK, &sh.kfull[s],
                              kb * 64, krow + tile * BN);
         issued = t + 1;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       // Let every copy this thread started land before the CTA can exit.
       sm100::mbar_wait(&sh.qfull, 0, kWaitLimitNs);
@@ -235,12 +463,14 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       const uint32_t ak = sm100::smem_u32(sK);
       int done = 0;
       if (wait_or_abort(&sh.qfull, 0, abort_flag, a.status)) {
+        int s = 0;
+        uint32_t ph = 0;
         for (int t = 0; t < TT; ++t) {
-          const int s = t % NS, buf = t & 1;
-          if (!wait_or_abort(&sh.kfull[s], (t / NS) & 1, abort_flag, a.status))
-            break;
-          if (t >= 2 && !wait_or_abort(&sh.tempty[buf], ((t >> 1) & 1) ^ 1,
-                                       abort_flag, a.status))
+          const int buf = t & (kTmemBufs - 1);
+          if (!wait_or_abort(&sh.kfull[s], ph, abort_flag, a.status)) break;
+          if (t >= kTmemBufs &&
+              !wait_or_abort(&sh.tempty[buf], ((t / kTmemBufs) & 1) ^ 1,
+                             abort_flag, a.status))
             break;
           sm100::tc_fence_after();
           const uint32_t d_tmem = tmem + buf * BN;
@@ -254,21 +484,43 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
           sm100::mma_commit(&sh.kempty[s]);
           sm100::mma_commit(&sh.tfull[buf]);
           done = t + 1;
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1;
+          }
         }
       }
       // The last commit covers every MMA issued: wait for it before exit.
       if (done > 0)
-        sm100::mbar_wait(&sh.tfull[(done - 1) & 1], ((done - 1) >> 1) & 1,
-                         kWaitLimitNs);
+        sm100::mbar_wait(&sh.tfull[(done - 1) & (kTmemBufs - 1)],
+                         ((done - 1) / kTmemBufs) & 1, kWaitLimitNs);
     }
   } else {
-    // ---------------- selector warps: thread = query row, group = chunk
+    // ---------------- selector warps: thread = (query row, chunk group)
     const int sw = warp - 2;               // 0..15
     const int grp = sw >> 2;               // 32-column chunk of every tile
     const int quarter = warp & 3;          // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
+    const int col = grp * kTileRows + r;   // this thread's segment column
     const int hi = sh.hi[r];
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + grp * 32;
+
+    // Scores of key tile t for this thread's row and chunk, with
+    // non-candidates (j = 0, the window, the future) replaced by NaN.
+    auto fetch = [&](int t, uint32_t (&raw)[32]) -> bool {
+      const int buf = t & (kTmemBufs - 1);
+      if (!__all_sync(0xFFFFFFFFu,
+                      wait_or_abort(&sh.tfull[buf], (t / kTmemBufs) & 1,
+                                    abort_flag, a.status)))
+        return false;
+      sm100::tc_fence_after();
+      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
+      sm100::tmem_wait_ld();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
+      return true;
+    };
 
     // ---- pass 1: slot maxima
     float colmax[32];
@@ -276,28 +528,17 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     for (int x = 0; x < 32; ++x) colmax[x] = -INFINITY;
     int t = 0;
     for (; t < T; ++t) {
-      const int buf = t & 1;
-      if (!__all_sync(0xFFFFFFFFu, wait_or_abort(&sh.tfull[buf], (t >> 1) & 1,
-                                                 abort_flag, a.status)))
-        break;
-      sm100::tc_fence_after();
       uint32_t raw[32];
-      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
-      sm100::tmem_wait_ld();
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
+      if (!fetch(t, raw)) break;
       const int j0 = t * BN + grp * 32;
-      if (__all_sync(0xFFFFFFFFu, j0 >= 1 && j0 + 31 <= hi)) {
+      if (!(j0 >= 1 && j0 + 31 <= hi)) {
 #pragma unroll
         for (int x = 0; x < 32; ++x)
-          colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
-      } else {
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (j0 + x >= 1 && j0 + x <= hi)
-            colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
+          if (!(j0 + x >= 1 && j0 + x <= hi)) raw[x] = kMaskedScore;
       }
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
     }
     // ---- bound: k-th largest of the row's 128 slot maxima.  The table
     // row is stored with its 16-byte pieces XOR-swizzled by the row index so
@@ -310,88 +551,121 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                       colmax[4 * c + 3]);
     }
     SelBar::sync();
-    for (int rr = 0; rr < 8; ++rr) {
-      const int row = sw * 8 + rr;
-      const int piece = lane ^ (row & 31);
-      const float4 v = *reinterpret_cast<const float4*>(table + row * 128 +
-                                                         piece * 4);
-      uint32_t key[4] = {ord_f32(v.x), ord_f32(v.y), ord_f32(v.z),
-                         ord_f32(v.w)};
-      warp_bitonic<4>(key, lane);  // ascending over 128 slots
-      const int e = 128 - k;       // the k-th largest
-      const uint32_t kk = __shfl_sync(0xFFFFFFFFu, key[e >> 5], e & 31);
-      if (lane == 0)
-        sh.L[row] = (kk <= ord_f32(-INFINITY)) ? -INFINITY : unord_f32(kk);
+    {
+      // Four lanes per row (part = slots part*32 .. part*32+31), eight rows
+      // per warp.  tau is the largest value with its low 14 bits zero and at
+      // least k slots >= tau (or the first probe that leaves exactly k); any
+      // such tau is a valid bound.
+      const int row = sw * 8 + (lane >> 2), part = lane & 3;
+      uint32_t key[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int piece = (part * 8 + c) ^ (row & 31);
+        const float4 v = *reinterpret_cast<const float4*>(table + row * 128 +
+                                                           piece * 4);
+        key[4 * c] = ord_f32(v.x);
+        key[4 * c + 1] = ord_f32(v.y);
+        key[4 * c + 2] = ord_f32(v.z);
+        key[4 * c + 3] = ord_f32(v.w);
+      }
+      uint32_t tau = 0u;
+      bool done = false;
+#pragma unroll 1
+      for (int bit = 31; bit >= 14; --bit) {
+        const uint32_t c = tau | (1u << bit);
+        int m = 0;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) m += key[x] >= c;
+        m = quad_sum(m);
+        const bool up = !done && m >= k;
+        tau = up ? c : tau;
+        done |= up && m == k;
+        if (__all_sync(0xFFFFFFFFu, done)) break;
+      }
+      if (part == 0)
+        sh.L[row] = (tau <= ord_f32(-INFINITY)) ? -INFINITY : unord_f32(tau);
     }
     SelBar::sync();
     const float Lr = sh.L[r];
-    bool ovf_local = false;
-    // ---- pass 2: append every candidate >= L
+    // ---- pass 2: append every candidate >= L to this thread's segment; a
+    // full segment continues in a spare one (rare), else the row is listed
+    // for the exact fallback.
+    const uint32_t seg_s = sm100::smem_u32(seg), seg_c = sm100::smem_u32(codes);
+    uint32_t as0 = seg_s + col * 4, ac0 = seg_c + col * 2;
+    // cursors are checked every 8 columns so that 8 more entries still fit
+    uint32_t as_max = as0 + (uint32_t)(P - 8) * kScoreStride;
+    uint32_t ac_max = ac0 + (uint32_t)(P - 8) * kCodeStride;
+    uint32_t as = as0, ac = ac0;
+    int xc = -1, own = 0;
+    bool ovf = false;
     for (; t < TT; ++t) {
-      const int buf = t & 1;
-      if (!__all_sync(0xFFFFFFFFu, wait_or_abort(&sh.tfull[buf], (t >> 1) & 1,
-                                                 abort_flag, a.status)))
-        break;
-      sm100::tc_fence_after();
       uint32_t raw[32];
-      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
-      sm100::tmem_wait_ld();
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
-      const int j0 = (t - T) * BN + grp * 32;
-      // A score can only qualify if it reaches L; one warp vote per column
-      // keeps the (rare) append off the common path.
-      auto append = [&](uint32_t bits, int j) {
-        const int pos = atomicAdd(&sh.cnt[r], 1);
-        if (pos < cap)
-          rbuf[(size_t)pos * kTileRows + r] = make_key(__uint_as_float(bits),
-                                                       (uint32_t)j);
-        else
-          ovf_local = true;
-      };
-      if (__all_sync(0xFFFFFFFFu, j0 >= 1 && j0 + 31 <= hi)) {
+      if (!fetch(t, raw)) break;
+      const int tile = t - T;
+      const int j0 = tile * BN + grp * 32;
+      if (!(j0 >= 1 && j0 + 31 <= hi)) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const bool p = __uint_as_float(raw[x]) >= Lr;
-          if (__any_sync(0xFFFFFFFFu, p)) {
-            if (p) append(raw[x], j0 + x);
+        for (int x = 0; x < 32; ++x)
+          if (!(j0 + x >= 1 && j0 + x <= hi)) raw[x] = kMaskedScore;
+      }
+      const uint32_t cbase = (uint32_t)tile * 32;
+      const uint32_t as_t = as;  // cursor at the tile start
+      bool full = false;
+      append_tile(raw, as, ac, Lr, cbase, as_max, ac_max, full);
+      if (__any_sync(0xFFFFFFFFu, full)) {
+        // An own segment is full: drop this tile's entries from it and redo
+        // the tile in a spare segment (once per thread, while any is left);
+        // otherwise the row goes to the exact fallback.  The whole warp runs
+        // the redo; threads with nothing to redo append nothing (L = +inf).
+        float Lredo = INFINITY;
+        if (full) {
+          const int px = (xc < 0 && !ovf) ? atomicAdd(&sh.pool, 1) : kPoolCols;
+          if (px < kPoolCols) {
+            own = (as_t - as0) / kScoreStride;
+            xc = px;
+            as0 = seg_s + (kSelThreads + px) * 4;
+            ac0 = seg_c + (kSelThreads + px) * 2;
+            as_max = as0 + (uint32_t)(P - 8) * kScoreStride;
+            ac_max = ac0 + (uint32_t)(P - 8) * kCodeStride;
+            as = as0;
+            ac = ac0;
+            Lredo = Lr;
+          } else {
+            ovf = true;
           }
         }
-      } else {
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const bool p = j0 + x >= 1 && j0 + x <= hi &&
-                         __uint_as_float(raw[x]) >= Lr;
-          if (__any_sync(0xFFFFFFFFu, p)) {
-            if (p) append(raw[x], j0 + x);
-          }
-        }
+        bool full2 = false;
+        append_tile(raw, as, ac, Lredo, cbase, as_max, ac_max, full2);
+        ovf |= full2;
       }
     }
-    if (ovf_local) sh.ovf[r] = 1;
+    const int last = (as - as0) / kScoreStride;
+    sh.cnt[col] = ovf ? (short)-1 : (short)(xc < 0 ? last : own);
+    sh.xcnt[col] = (short)(xc < 0 ? 0 : last);
+    sh.xcol[col] = (signed char)xc;
     SelBar::sync();
-    // ---- exact Top-k of the row's buffer (one thread per row)
-    if (grp == 0) {
-      const int i = i0 + r;
-      if (i < a.n && k > 0) {
-        const size_t grow = (size_t)(b * a.Hq + h) * a.n + i;
-        uint64_t* out = a.topk + grow * k;
-        if (sh.ovf[r]) {
-          // listed for the exact fallback pass; it writes this row
+    // ---- exact Top-k per row: four lanes per row, eight rows per warp
+    {
+      const int row = sw * 8 + (lane >> 2), part = lane & 3;
+      const int i = i0 + row;
+      RowSegs rs;
+      row_segs(sh, row, rs);
+      const size_t grow = (size_t)(b * a.Hq + h) * a.n + i;
+      bool live = i < a.n;
+      if (live && (rs.bad || rs.n > 128)) {
+        // listed for the exact fallback pass; it writes this row
+        if (part == 0) {
           const uint32_t pos = atomicAdd(a.ovf_count, 1u);
           a.ovf_rows[pos] = (uint32_t)grow;
-        } else {
-          for (int e = 0; e < k; ++e) heap[e * kTileRows + r] = 0ull;
-          uint64_t root = 0ull;
-          const int n = sh.cnt[r];
-          for (int e = 0; e < n; ++e) {
-            const uint64_t key = rbuf[(size_t)e * kTileRows + r];
-            if (key > root) root = heap_replace(heap, k, r, key);
-          }
-          for (int e = 0; e < k; ++e) out[e] = heap[e * kTileRows + r];
         }
+        live = false;
       }
+      const uint32_t lob = ord_f32(sh.L[row]);
+      uint64_t* out = a.topk + grow * k;
+      if (__all_sync(0xFFFFFFFFu, !live || rs.n <= 64))
+        quad_select<16>(seg, codes, rs, live, lob, k, out, part);
+      else
+        quad_select<32>(seg, codes, rs, live, lob, k, out, part);
     }
   }
   __syncwarp();  // reconverge single-lane roles before the CTA barrier
@@ -399,7 +673,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   __syncthreads();
   if (warp == 1) {
     sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, 256);
+    sm100::tmem_dealloc(tmem, kTmemBufs * BN);
   }
 }
 
@@ -746,29 +1020,31 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int d) {
 template <int D>
 cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   using Lay = TcLayout<D>;
+  // segment codes hold tile * 32 + column in 16 bits
+  if ((a.n + Lay::BN - 1) / Lay::BN > 2048) return cudaErrorNotSupported;
   CUtensorMap tq, tk;
   if (!make_tmap(&tq, a.Q, (uint64_t)a.B * a.Hq * a.n, D)) return cudaErrorInvalidValue;
   if (!make_tmap(&tk, a.K, (uint64_t)a.B * a.Hkv * a.n, D)) return cudaErrorInvalidValue;
-  // row buffer: 3k candidates (the pass-1 bound leaves about 1.1-1.4 k),
-  // at least kMinCap slots, at most what fits next to Q and the K ring
+  // Segment positions per (row, chunk group) thread: about k/4 entries are
+  // expected (1.1-1.4 k per row), but one key tile can put 31 entries into
+  // one segment (rows with fewer than k candidates); the cursor check every
+  // 8 columns keeps 8 positions in reserve.
   const size_t budget = 227 * 1024 - sizeof(TcShared);
-  const int cap_max = (int)((budget - Lay::bytes(0)) / (kTileRows * 8));
-  int cap = 3 * a.k;
-  if (cap < kMinCap) cap = kMinCap;
-  if (cap > cap_max) cap = cap_max;
-  if (cap < a.k || cap < kMinCap) return cudaErrorNotSupported;
-  const size_t smem = Lay::bytes(cap);
+  int P = a.k > 32 ? 46 : 40;
+  while (P > kMinSeg && Lay::bytes(P) > budget) --P;
+  if (Lay::bytes(P) > budget || P < 40) return cudaErrorNotSupported;
+  const size_t smem = Lay::bytes(P);
   auto kern = prefill_score_topk_tc<D>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_tc");
-  kern<<<grid, kTcThreads, smem, s>>>(tq, tk, a, cap);
+  kern<<<grid, kTcThreads, smem, s>>>(tq, tk, a, P);
   prof_after(s);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // rows whose buffer overflowed (none on typical inputs): exact fallback
+  // rows whose segments overflowed (rare on typical inputs): exact fallback
   const size_t fb_smem = (size_t)(a.k + kFbChunk) * 8 + D * 4;
   prof_before(s, "prefill_overflow_rows");
   prefill_overflow_rows<__nv_bfloat16, D><<<148, kFbThreads, fb_smem, s>>>(a);
