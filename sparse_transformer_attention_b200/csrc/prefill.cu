@@ -32,7 +32,6 @@ namespace ca {
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
-constexpr int kGatherThreads = 256;
 
 // ------------------------------------------------------------ shared prologue
 // Window and last candidate position of each row of the tile; returns the
@@ -842,22 +841,69 @@ __device__ __forceinline__ void warp_sort(uint32_t (&v)[NPL], int lane) {
   }
 }
 
+// Raw (undecoded) copy of DL consecutive elements of a row.
+template <typename T, int DL>
+struct RawRow {
+  static constexpr int kWords = DL * (int)sizeof(T) / 16;  // 16-byte pieces
+  uint4 w[kWords];
+  __device__ __forceinline__ void load(const T* p) {
+    const uint4* s = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int c = 0; c < kWords; ++c) w[c] = __ldg(s + c);
+  }
+  __device__ __forceinline__ void to_f32(float (&f)[DL]) const {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int c = 0; c < kWords; ++c) {
+        f[8 * c + 0] = bf16lo(w[c].x);
+        f[8 * c + 1] = bf16hi(w[c].x);
+        f[8 * c + 2] = bf16lo(w[c].y);
+        f[8 * c + 3] = bf16hi(w[c].y);
+        f[8 * c + 4] = bf16lo(w[c].z);
+        f[8 * c + 5] = bf16hi(w[c].z);
+        f[8 * c + 6] = bf16lo(w[c].w);
+        f[8 * c + 7] = bf16hi(w[c].w);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kWords; ++c) {
+        f[4 * c + 0] = __uint_as_float(w[c].x);
+        f[4 * c + 1] = __uint_as_float(w[c].y);
+        f[4 * c + 2] = __uint_as_float(w[c].z);
+        f[4 * c + 3] = __uint_as_float(w[c].w);
+      }
+    }
+  }
+};
+
+// Four query rows per warp, eight lanes per row (each lane holds D/8 head
+// dimensions of q, of the output and of every K and V row it reads).
+//   1. For each row, with the whole warp: sort the Top-k positions and write
+//      C_i (ascending, -1 padded) and |C_i|.
+//   2. fp32 softmax over C_i, KPC keys at a time: the K and V loads of a
+//      chunk are issued together, then the chunk's scores (Top-k scores come
+//      with the keys, anchor and window scores are dot products reduced over
+//      the row's eight lanes) move the running maximum once.  Window rows are
+//      shared by the warp's neighbouring queries, so they mostly hit L1.
+constexpr int kGatherWarps = 8;
+constexpr int kGatherRPW = 4;              // rows per warp
+constexpr int kGatherLPR = 32 / kGatherRPW;  // lanes per row
+
 template <typename T, int D, typename TO, int NPL>
-__global__ void __launch_bounds__(kGatherThreads)
+__global__ void __launch_bounds__(kGatherWarps * 32)
 prefill_gather(PrefillArgs a) {
-  constexpr int LPR = 4;          // lanes per row in the softmax
-  constexpr int RPW = 32 / LPR;   // rows per warp
-  constexpr int DL = D / LPR;     // head dims per lane
-  const int lane = threadIdx.x & 31;
-  const int64_t wglob = ((int64_t)blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
+  constexpr int DL = D / kGatherLPR;
+  constexpr int KPC = 4;  // keys per chunk
+  __shared__ uint64_t s_key[kGatherWarps][kGatherRPW][kPrefillMaxK];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t R = (int64_t)a.B * a.Hq * a.n;
-  const int64_t row0 = wglob * RPW;
-  if (row0 >= R) return;
+  const int64_t row0 = ((int64_t)blockIdx.x * kGatherWarps + wid) * kGatherRPW;
+  if (row0 >= R) return;  // the whole warp
   const int k = a.k;
 
-  // ---- phase 1: one row at a time across the warp: sort, write C_i
+  // ---- 1: C_i, one row at a time across the warp
 #pragma unroll 1
-  for (int rr = 0; rr < RPW; ++rr) {
+  for (int rr = 0; rr < kGatherRPW; ++rr) {
     const int64_t row = row0 + rr;
     if (row >= R) break;
     const int64_t bh = row / a.n;
@@ -874,6 +920,7 @@ prefill_gather(PrefillArgs a) {
       const int e = t * 32 + lane;
       uint64_t key = 0ull;
       if (e < k) key = a.topk[row * k + e];
+      if (e < k) s_key[wid][rr][e] = key;
       v[t] = key ? key_index(key) : 0xFFFFFFFFu;
       m += __popc(__ballot_sync(0xFFFFFFFFu, key != 0ull));
     }
@@ -903,10 +950,11 @@ prefill_gather(PrefillArgs a) {
     }
     if (lane == 0) a.idx_count[row] = count;
   }
+  __syncwarp();
 
-  // ---- phase 2: LPR lanes per row, fp32 online softmax over C_i
-  const int sub = lane % LPR;
-  const int64_t row = row0 + lane / LPR;
+  // ---- 2: softmax over C_i, eight lanes per row
+  const int rloc = lane / kGatherLPR, sub = lane % kGatherLPR;
+  const int64_t row = row0 + rloc;
   const bool live = row < R;
   const int64_t rowc = live ? row : R - 1;
   const int64_t bh = rowc / a.n;
@@ -916,67 +964,103 @@ prefill_gather(PrefillArgs a) {
   const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n, a.status,
                            false);
   const int lo = i - w + 1 > 0 ? i - w + 1 : 0;
-  const T* qp = reinterpret_cast<const T*>(a.Q) + rowc * D + sub * DL;
+  const int anc = lo > 0 ? 1 : 0;
   const T* Kg = reinterpret_cast<const T*>(a.K) +
                 ((size_t)b * a.Hkv + g) * a.n * D + sub * DL;
   const T* Vg = reinterpret_cast<const T*>(a.V) +
                 ((size_t)b * a.Hkv + g) * a.n * D + sub * DL;
   float qv[DL];
-#pragma unroll
-  for (int e = 0; e < DL; e += 4) load_f32<T, 4>(qp + e, qv + e);
+  {
+    RawRow<T, DL> qr;
+    qr.load(reinterpret_cast<const T*>(a.Q) + rowc * D + sub * DL);
+    qr.to_f32(qv);
+  }
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);
-  float mx = -INFINITY, den = 0.f, o[DL];
+  float mrun = -INFINITY, den = 0.f, o[DL];
 #pragma unroll
   for (int e = 0; e < DL; ++e) o[e] = 0.f;
 
-  auto accumulate = [&](float s_scaled, const T* vrow) {
-    float vf[DL];
+  // fold a chunk of scores s[u] (log2 units; -inf = no key) and V rows
+  auto fold = [&](const float (&s)[KPC], const RawRow<T, DL> (&vr)[KPC]) {
+    float cm = s[0];
 #pragma unroll
-    for (int e = 0; e < DL; e += 4) load_f32<T, 4>(vrow + e, vf + e);
-    const float mn = fmaxf(mx, s_scaled);
-    const float corr = exp2f(mx - mn);
-    const float p = exp2f(s_scaled - mn);
-    den = den * corr + p;
+    for (int u = 1; u < KPC; ++u) cm = fmaxf(cm, s[u]);
+    if (cm == -INFINITY) return;  // uniform over the row's lanes
+    const float mn = fmaxf(mrun, cm);
+    const float sc = exp2f(mrun - mn);
+    den *= sc;
 #pragma unroll
-    for (int e = 0; e < DL; ++e) o[e] = fmaf(p, vf[e], o[e] * corr);
-    mx = mn;
+    for (int e = 0; e < DL; ++e) o[e] *= sc;
+#pragma unroll
+    for (int u = 0; u < KPC; ++u) {
+      const float p = exp2f(s[u] - mn);  // 0 for s = -inf
+      float vf[DL];
+      vr[u].to_f32(vf);
+      den += p;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) o[e] = fmaf(p, vf[e], o[e]);
+    }
+    mrun = mn;
   };
 
-  // Top-k entries: scores come with the keys (the selector's fp32 values)
-  const uint64_t* tk = a.topk + rowc * k;
-#pragma unroll 1
-  for (int e = 0; e < k; ++e) {
-    const uint64_t key = live ? tk[e] : 0ull;
-    if (key == 0ull) continue;
-    const uint32_t j = key_index(key);
-    if (j == 0 || (int)j > i - w) {  // never written by the selector
-      raise_flag(a.status, kErrInternal);
-      continue;
+  // Top-k entries: the selector's fp32 scores
+  for (int c0 = 0; c0 < k; c0 += KPC) {
+    float s[KPC];
+    RawRow<T, DL> vr[KPC];
+#pragma unroll
+    for (int u = 0; u < KPC; ++u) {
+      const int e = c0 + u;
+      const uint64_t key = (live && e < k) ? s_key[wid][rloc][e] : 0ull;
+      uint32_t j = key ? key_index(key) : 0u;
+      bool act = key != 0ull;
+      if (act && (j == 0 || (int)j > i - w)) {  // never written by the selector
+        raise_flag(a.status, kErrInternal);
+        act = false;
+        j = 0;
+      }
+      s[u] = act ? key_score(key) * sl2 : -INFINITY;
+      vr[u].load(Vg + (size_t)j * D);
     }
-    accumulate(key_score(key) * sl2, Vg + (size_t)j * D);
+    fold(s, vr);
   }
-  // anchor and window: scores computed here, 4 lanes per dot product
-  const int nw = live ? (i - lo + 1) + (lo > 0 ? 1 : 0) : 0;
+  // anchor and window: dot products over the row's eight lanes
+  const int nw = live ? anc + (i - lo + 1) : 0;
   int nmax = nw;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1)
     nmax = max(nmax, __shfl_xor_sync(0xFFFFFFFFu, nmax, off));
-#pragma unroll 1
-  for (int t = 0; t < nmax; ++t) {
-    const bool act = t < nw;
-    int j = 0;
-    if (lo > 0) j = (t == 0) ? 0 : lo + t - 1;
-    else j = lo + t;
-    if (!act) j = 0;
-    float kf[DL];
+  for (int c0 = 0; c0 < nmax; c0 += KPC) {
+    RawRow<T, DL> kr[KPC], vr[KPC];
+    int jj[KPC];
 #pragma unroll
-    for (int e = 0; e < DL; e += 4) load_f32<T, 4>(Kg + (size_t)j * D + e, kf + e);
-    float dot = 0.f;
+    for (int u = 0; u < KPC; ++u) {
+      const int li = c0 + u;
+      jj[u] = li < nw ? ((anc && li == 0) ? 0 : lo + li - anc) : 0;
+      kr[u].load(Kg + (size_t)jj[u] * D);
+      vr[u].load(Vg + (size_t)jj[u] * D);
+    }
+    float s[KPC];
 #pragma unroll
-    for (int e = 0; e < DL; ++e) dot = fmaf(qv[e], kf[e], dot);
-    dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
-    dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 2);
-    if (act) accumulate(dot * sl2, Vg + (size_t)j * D);
+    for (int u = 0; u < KPC; ++u) {
+      float kf[DL];
+      kr[u].to_f32(kf);
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; e += 2) {
+        d0 = fmaf(qv[e], kf[e], d0);
+        d1 = fmaf(qv[e + 1], kf[e + 1], d1);
+      }
+      s[u] = d0 + d1;
+    }
+#pragma unroll
+    for (int off = kGatherLPR / 2; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < KPC; ++u)
+        s[u] += __shfl_xor_sync(0xFFFFFFFFu, s[u], off);
+#pragma unroll
+    for (int u = 0; u < KPC; ++u)
+      s[u] = (c0 + u < nw) ? s[u] * sl2 : -INFINITY;
+    fold(s, vr);
   }
   if (live) {
     TO* op = reinterpret_cast<TO*>(a.O) + rowc * D + sub * DL;
@@ -1070,16 +1154,16 @@ cudaError_t launch_select_f32(const PrefillArgs& a, cudaStream_t s) {
 template <typename T, int D>
 cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
   const int64_t R = (int64_t)a.B * a.Hq * a.n;
-  const int64_t warps = (R + 7) / 8;
-  const int64_t blocks = (warps * 32 + kGatherThreads - 1) / kGatherThreads;
-  dim3 grid((unsigned)blocks);
+  const int64_t rows_per_cta = (int64_t)kGatherWarps * kGatherRPW;
+  dim3 grid((unsigned)((R + rows_per_cta - 1) / rows_per_cta));
+  const int nt = kGatherWarps * 32;
   prof_before(s, "prefill_gather");
   if (a.k <= 32) {
-    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 1><<<grid, kGatherThreads, 0, s>>>(a);
-    else prefill_gather<T, D, float, 1><<<grid, kGatherThreads, 0, s>>>(a);
+    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 1><<<grid, nt, 0, s>>>(a);
+    else prefill_gather<T, D, float, 1><<<grid, nt, 0, s>>>(a);
   } else {
-    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 2><<<grid, kGatherThreads, 0, s>>>(a);
-    else prefill_gather<T, D, float, 2><<<grid, kGatherThreads, 0, s>>>(a);
+    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 2><<<grid, nt, 0, s>>>(a);
+    else prefill_gather<T, D, float, 2><<<grid, nt, 0, s>>>(a);
   }
   prof_after(s);
   return cudaGetLastError();
