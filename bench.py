@@ -308,7 +308,10 @@ def run_ours(args, rank, world, local_rank):
     launches = len(prof)  # library kernels launched per timed pass
     pk = peaks()
     model = work_model(w)
-    dom = max(kern_avg, key=lambda k_: sum(per[k_]))
+    # the dominant kernel among those with a work model (the exact fallback
+    # for overflowing prefill rows has none: its work depends on the rows)
+    dom = max((k_ for k_ in kern_avg if k_ in model),
+              key=lambda k_: sum(per[k_]))
     bound, work, what = model[dom]
     t_dom = kern_avg[dom] * 1e-3
     if bound == "tensor":

@@ -676,6 +676,41 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   }
 }
 
+// Raw (undecoded) copy of DL consecutive elements of a row.
+template <typename T, int DL>
+struct RawRow {
+  static constexpr int kWords = DL * (int)sizeof(T) / 16;  // 16-byte pieces
+  uint4 w[kWords];
+  __device__ __forceinline__ void load(const T* p) {
+    const uint4* s = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int c = 0; c < kWords; ++c) w[c] = __ldg(s + c);
+  }
+  __device__ __forceinline__ void to_f32(float (&f)[DL]) const {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int c = 0; c < kWords; ++c) {
+        f[8 * c + 0] = bf16lo(w[c].x);
+        f[8 * c + 1] = bf16hi(w[c].x);
+        f[8 * c + 2] = bf16lo(w[c].y);
+        f[8 * c + 3] = bf16hi(w[c].y);
+        f[8 * c + 4] = bf16lo(w[c].z);
+        f[8 * c + 5] = bf16hi(w[c].z);
+        f[8 * c + 6] = bf16lo(w[c].w);
+        f[8 * c + 7] = bf16hi(w[c].w);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kWords; ++c) {
+        f[4 * c + 0] = __uint_as_float(w[c].x);
+        f[4 * c + 1] = __uint_as_float(w[c].y);
+        f[4 * c + 2] = __uint_as_float(w[c].z);
+        f[4 * c + 3] = __uint_as_float(w[c].w);
+      }
+    }
+  }
+};
+
 // Exact fallback for rows whose candidate buffer overflowed: one CTA per
 // listed row scores every candidate on CUDA cores (fp32 FMA of the bf16 or
 // fp32 inputs) and keeps the best k keys with the CTA radix select.
@@ -710,10 +745,18 @@ prefill_overflow_rows(PrefillArgs a) {
     for (int c0 = 1; c0 <= hi; c0 += kFbChunk) {
       for (int jj = threadIdx.x; jj < kFbChunk && c0 + jj <= hi; jj += kFbThreads) {
         const int j = c0 + jj;
-        const T* kr = Kg + (size_t)j * D;
-        float acc = 0.f;
-        for (int e = 0; e < D; ++e) acc = fmaf(q[e], Elem<T>::load1(kr + e), acc);
-        keys[s_n + jj] = make_key(acc, (uint32_t)j);
+        // the key row in 16-byte pieces, all loads issued before the FMAs
+        RawRow<T, D> kr;
+        kr.load(Kg + (size_t)j * D);
+        float kf[D];
+        kr.to_f32(kf);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < D; e += 2) {
+          a0 = fmaf(q[e], kf[e], a0);
+          a1 = fmaf(q[e + 1], kf[e + 1], a1);
+        }
+        keys[s_n + jj] = make_key(a0 + a1, (uint32_t)j);
       }
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -840,41 +883,6 @@ __device__ __forceinline__ void warp_sort(uint32_t (&v)[NPL], int lane) {
     }
   }
 }
-
-// Raw (undecoded) copy of DL consecutive elements of a row.
-template <typename T, int DL>
-struct RawRow {
-  static constexpr int kWords = DL * (int)sizeof(T) / 16;  // 16-byte pieces
-  uint4 w[kWords];
-  __device__ __forceinline__ void load(const T* p) {
-    const uint4* s = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-    for (int c = 0; c < kWords; ++c) w[c] = __ldg(s + c);
-  }
-  __device__ __forceinline__ void to_f32(float (&f)[DL]) const {
-    if constexpr (sizeof(T) == 2) {
-#pragma unroll
-      for (int c = 0; c < kWords; ++c) {
-        f[8 * c + 0] = bf16lo(w[c].x);
-        f[8 * c + 1] = bf16hi(w[c].x);
-        f[8 * c + 2] = bf16lo(w[c].y);
-        f[8 * c + 3] = bf16hi(w[c].y);
-        f[8 * c + 4] = bf16lo(w[c].z);
-        f[8 * c + 5] = bf16hi(w[c].z);
-        f[8 * c + 6] = bf16lo(w[c].w);
-        f[8 * c + 7] = bf16hi(w[c].w);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < kWords; ++c) {
-        f[4 * c + 0] = __uint_as_float(w[c].x);
-        f[4 * c + 1] = __uint_as_float(w[c].y);
-        f[4 * c + 2] = __uint_as_float(w[c].z);
-        f[4 * c + 3] = __uint_as_float(w[c].w);
-      }
-    }
-  }
-};
 
 // Four query rows per warp, eight lanes per row (each lane holds D/8 head
 // dimensions of q, of the output and of every K and V row it reads).
