@@ -1078,6 +1078,344 @@ prefill_gather(PrefillArgs a) {
   }
 }
 
+// ------------------------------------------------- tensor-core window part
+// Warp-level MMA (mma.sync) on the banded window scores: 16 query rows per
+// warp against 16-key blocks of the rows' window span.  Scores: m16n8k16 with
+// bf16 Q and K, fp32 accumulation (exact products, like the CUDA-core dot).
+// p * V: m16n8k8 with tf32 p (rounded from fp32, 11 significant bits) and V
+// (bf16 widened exactly), so the weights keep more precision than bf16.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4],
+                                               const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], uint32_t a0,
+                                              uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16* p) {
+  return __ldg(reinterpret_cast<const unsigned int*>(p));
+}
+__device__ __forceinline__ uint32_t bf16_bits_as_f32(const __nv_bfloat16* p) {
+  return (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16;
+}
+
+constexpr int kMmaWarps = 4;  // 16 query rows each
+
+// Per warp: the window state (o, max, sum) of its 16 rows, then their Top-k
+// keys as read in step 1.
+template <int D>
+struct MmaGatherSmem {
+  static constexpr size_t state = (size_t)16 * D * 4 + 2 * 16 * 4;
+  __host__ __device__ static size_t per_warp(int k) {
+    return state + (size_t)16 * k * 8;
+  }
+  __host__ __device__ static size_t bytes(int k) { return kMmaWarps * per_warp(k); }
+};
+
+// bf16 gather with the window on tensor cores.  A warp owns 16 consecutive
+// query rows of one (batch, head).
+//   1. C_i and |C_i| for each of its rows (whole warp per row).
+//   2. The window [lo_i, i] of all 16 rows: MMA scores, masked per row, an
+//      online softmax per row over 16-key blocks, and the MMA p * V.  The
+//      state (max, sum, unnormalised o) goes to shared memory.
+//   3. Eight lanes per row, four rows at a time: start from the window state
+//      and fold in the Top-k keys (scores from the selector) and the anchor
+//      (score computed here), then write the output row.
+template <int D, typename TO, int NPL>
+__global__ void __launch_bounds__(kMmaWarps * 32)
+prefill_gather_mma(PrefillArgs a) {
+  using T = __nv_bfloat16;
+  constexpr int KS = D / 16;  // k-steps of the score MMA
+  constexpr int NT = D / 8;   // head-dim tiles of the p * V MMA
+  extern __shared__ __align__(16) unsigned char g_smem[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int n = a.n, k = a.k;
+  float* s_o = reinterpret_cast<float*>(g_smem + wid * MmaGatherSmem<D>::per_warp(k));
+  float* s_m = s_o + 16 * D;
+  float* s_l = s_m + 16;
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_l + 16);  // [16][k]
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int g = h / (a.Hq / a.Hkv);
+  const int i0 = (blockIdx.x * kMmaWarps + wid) * 16;
+  if (i0 >= n) return;  // the whole warp
+  const int64_t rowbase = (int64_t)bh * n;
+  const T* Qg = reinterpret_cast<const T*>(a.Q) + rowbase * D;
+  const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * n * D;
+  const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * n * D;
+
+  // ---- 1: C_i, one row at a time across the warp
+#pragma unroll 1
+  for (int rr = 0; rr < 16; ++rr) {
+    const int i = i0 + rr;
+    if (i >= n) break;
+    const int64_t row = rowbase + i;
+    const int w = row_window(a.W_i, (int64_t)b * n + i, a.W, n, a.status, false);
+    const int lo = i - w + 1 > 0 ? i - w + 1 : 0;
+    const int anc = lo > 0 ? 1 : 0;
+    uint32_t v[NPL];
+    int m = 0;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      const int e = t * 32 + lane;
+      const uint64_t key = e < k ? a.topk[row * k + e] : 0ull;
+      if (e < k) s_key[rr * k + e] = key;
+      v[t] = key ? key_index(key) : 0xFFFFFFFFu;
+      m += __popc(__ballot_sync(0xFFFFFFFFu, key != 0ull));
+    }
+    warp_sort<NPL>(v, lane);
+    const int count = anc + m + (i - lo + 1);
+    if (count > a.C_max && lane == 0) raise_flag(a.status, kErrCmax);
+    const int wcount = count < a.C_max ? count : a.C_max;
+    int32_t* out = a.idx + row * a.C_max;
+    for (int rb = 0; rb < a.C_max; rb += 32) {
+      const int rpos = rb + lane;
+      const int tk = rpos - anc;
+      uint32_t sv = 0;
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) {
+        const uint32_t x = __shfl_sync(0xFFFFFFFFu, v[t], tk & 31);
+        if ((tk >> 5) == t) sv = x;
+      }
+      if (rpos < a.C_max) {
+        int32_t val;
+        if (rpos >= wcount) val = -1;
+        else if (rpos < anc) val = 0;
+        else if (tk < m) val = (int32_t)sv;
+        else val = lo + (tk - m);
+        out[rpos] = val;
+      }
+    }
+    if (lane == 0) a.idx_count[row] = count;
+  }
+
+  // ---- 2: window on tensor cores
+  const float sl2 = 1.4426950408889634f / sqrtf((float)D);
+  const int gr = lane >> 2, tq = lane & 3;  // fragment row group, thread in group
+  const int ia = i0 + gr, ib = i0 + gr + 8;  // this lane's two rows
+  const bool va = ia < n, vb = ib < n;
+  const int ca = va ? ia : n - 1, cb = vb ? ib : n - 1;
+  const int wa = row_window(a.W_i, (int64_t)b * n + ca, a.W, n, a.status, false);
+  const int wb = row_window(a.W_i, (int64_t)b * n + cb, a.W, n, a.status, false);
+  const int loa = ca - wa + 1 > 0 ? ca - wa + 1 : 0;
+  const int lob = cb - wb + 1 > 0 ? cb - wb + 1 : 0;
+  int kmin = min(loa, lob);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, off));
+  const int kmax = min(i0 + 15, n - 1);
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int c = 16 * ks + 2 * tq;
+    qa[ks][0] = ld_b32(Qg + (size_t)ca * D + c);
+    qa[ks][1] = ld_b32(Qg + (size_t)cb * D + c);
+    qa[ks][2] = ld_b32(Qg + (size_t)ca * D + c + 8);
+    qa[ks][3] = ld_b32(Qg + (size_t)cb * D + c + 8);
+  }
+  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+  float o[NT][4];
+#pragma unroll
+  for (int nd = 0; nd < NT; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+
+#pragma unroll 1
+  for (int j0 = kmin & ~15; j0 <= kmax; j0 += 16) {
+    float s[2][4];
+#pragma unroll
+    for (int h8 = 0; h8 < 2; ++h8) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int krow = min(j0 + 8 * h8 + gr, n - 1);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c = 16 * ks + 2 * tq;
+        mma_bf16_16816(acc, qa[ks], ld_b32(Kg + (size_t)krow * D + c),
+                       ld_b32(Kg + (size_t)krow * D + c + 8));
+      }
+      const int kc = j0 + 8 * h8 + 2 * tq;  // key of acc[0] / acc[2]
+      s[h8][0] = (va && kc >= loa && kc <= ia) ? acc[0] * sl2 : -INFINITY;
+      s[h8][1] = (va && kc + 1 >= loa && kc + 1 <= ia) ? acc[1] * sl2 : -INFINITY;
+      s[h8][2] = (vb && kc >= lob && kc <= ib) ? acc[2] * sl2 : -INFINITY;
+      s[h8][3] = (vb && kc + 1 >= lob && kc + 1 <= ib) ? acc[3] * sl2 : -INFINITY;
+    }
+    float xa = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+    float xb = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+    xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 1));
+    xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 2));
+    xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 1));
+    xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 2));
+    const float na = fmaxf(ma, xa), nb = fmaxf(mb, xb);
+    const float sa = na == -INFINITY ? 1.f : exp2f(ma - na);
+    const float sb = nb == -INFINITY ? 1.f : exp2f(mb - nb);
+    la *= sa;
+    lb *= sb;
+#pragma unroll
+    for (int nd = 0; nd < NT; ++nd) {
+      o[nd][0] *= sa;
+      o[nd][1] *= sa;
+      o[nd][2] *= sb;
+      o[nd][3] *= sb;
+    }
+    uint32_t p[2][4];
+#pragma unroll
+    for (int h8 = 0; h8 < 2; ++h8) {
+      const float p0 = s[h8][0] == -INFINITY ? 0.f : exp2f(s[h8][0] - na);
+      const float p1 = s[h8][1] == -INFINITY ? 0.f : exp2f(s[h8][1] - na);
+      const float p2 = s[h8][2] == -INFINITY ? 0.f : exp2f(s[h8][2] - nb);
+      const float p3 = s[h8][3] == -INFINITY ? 0.f : exp2f(s[h8][3] - nb);
+      p[h8][0] = to_tf32(p0);
+      p[h8][1] = to_tf32(p1);
+      p[h8][2] = to_tf32(p2);
+      p[h8][3] = to_tf32(p3);
+      // the sums use the rounded weights, as the MMA does
+      la += __uint_as_float(p[h8][0]) + __uint_as_float(p[h8][1]);
+      lb += __uint_as_float(p[h8][2]) + __uint_as_float(p[h8][3]);
+    }
+    // p * V, keys of the k8 step ordered (2t, 2t+1) -> (t, t+4) so that the
+    // score fragment is the A fragment as it stands
+#pragma unroll
+    for (int h8 = 0; h8 < 2; ++h8) {
+      const int kv0 = min(j0 + 8 * h8 + 2 * tq, n - 1);
+      const int kv1 = min(j0 + 8 * h8 + 2 * tq + 1, n - 1);
+#pragma unroll
+      for (int nd = 0; nd < NT; ++nd) {
+        const uint32_t b0 = bf16_bits_as_f32(Vg + (size_t)kv0 * D + 8 * nd + gr);
+        const uint32_t b1 = bf16_bits_as_f32(Vg + (size_t)kv1 * D + 8 * nd + gr);
+        mma_tf32_1688(o[nd], p[h8][0], p[h8][2], p[h8][1], p[h8][3], b0, b1);
+      }
+    }
+    ma = na;
+    mb = nb;
+  }
+  la += __shfl_xor_sync(0xFFFFFFFFu, la, 1);
+  la += __shfl_xor_sync(0xFFFFFFFFu, la, 2);
+  lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 1);
+  lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 2);
+  if (tq == 0) {
+    s_m[gr] = ma;
+    s_m[gr + 8] = mb;
+    s_l[gr] = la;
+    s_l[gr + 8] = lb;
+  }
+#pragma unroll
+  for (int nd = 0; nd < NT; ++nd) {
+    *reinterpret_cast<float2*>(s_o + gr * D + 8 * nd + 2 * tq) =
+        make_float2(o[nd][0], o[nd][1]);
+    *reinterpret_cast<float2*>(s_o + (gr + 8) * D + 8 * nd + 2 * tq) =
+        make_float2(o[nd][2], o[nd][3]);
+  }
+  __syncwarp();
+
+  // ---- 3: Top-k keys and the anchor, eight lanes per row
+  constexpr int DL = D / 8;
+  constexpr int KPC = 4;
+  const int sub = lane & 7, rq = lane >> 3;
+#pragma unroll 1
+  for (int rg = 0; rg < 4; ++rg) {
+    const int r = rg * 4 + rq;
+    const int i = i0 + r;
+    const bool live = i < n;
+    const int ic = live ? i : n - 1;
+    const int64_t row = rowbase + ic;
+    const int w = row_window(a.W_i, (int64_t)b * n + ic, a.W, n, a.status, false);
+    const int lo = ic - w + 1 > 0 ? ic - w + 1 : 0;
+    float mrun = s_m[r], den = s_l[r], ov[DL];
+#pragma unroll
+    for (int e = 0; e < DL; ++e) ov[e] = s_o[r * D + sub * DL + e];
+    float qv[DL];
+    {
+      RawRow<T, DL> qr;
+      qr.load(Qg + (size_t)ic * D + sub * DL);
+      qr.to_f32(qv);
+    }
+    auto fold = [&](const float (&sc)[KPC], const RawRow<T, DL> (&vr)[KPC]) {
+      float cm = sc[0];
+#pragma unroll
+      for (int u = 1; u < KPC; ++u) cm = fmaxf(cm, sc[u]);
+      if (cm == -INFINITY) return;  // uniform over the row's lanes
+      const float mn = fmaxf(mrun, cm);
+      const float f = exp2f(mrun - mn);
+      den *= f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) ov[e] *= f;
+#pragma unroll
+      for (int u = 0; u < KPC; ++u) {
+        const float pw = exp2f(sc[u] - mn);
+        float vf[DL];
+        vr[u].to_f32(vf);
+        den += pw;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) ov[e] = fmaf(pw, vf[e], ov[e]);
+      }
+      mrun = mn;
+    };
+    const T* Vs = Vg + sub * DL;
+    for (int c0 = 0; c0 < k; c0 += KPC) {
+      float sc[KPC];
+      RawRow<T, DL> vr[KPC];
+#pragma unroll
+      for (int u = 0; u < KPC; ++u) {
+        const int e = c0 + u;
+        const uint64_t key = (live && e < k) ? s_key[r * k + e] : 0ull;
+        uint32_t j = key ? key_index(key) : 0u;
+        bool act = key != 0ull;
+        if (act && (j == 0 || (int)j > ic - w)) {  // never written by the selector
+          raise_flag(a.status, kErrInternal);
+          act = false;
+          j = 0;
+        }
+        sc[u] = act ? key_score(key) * sl2 : -INFINITY;
+        vr[u].load(Vs + (size_t)j * D);
+      }
+      fold(sc, vr);
+    }
+    // the anchor (position 0) when it lies outside the window
+    {
+      float sc[KPC];
+      RawRow<T, DL> vr[KPC];
+      RawRow<T, DL> kr;
+      kr.load(Kg + sub * DL);
+      float kf[DL];
+      kr.to_f32(kf);
+      float d0 = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) d0 = fmaf(qv[e], kf[e], d0);
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1)
+        d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, off);
+      sc[0] = (live && lo > 0) ? d0 * sl2 : -INFINITY;
+      vr[0].load(Vs);
+#pragma unroll
+      for (int u = 1; u < KPC; ++u) {
+        sc[u] = -INFINITY;
+        vr[u] = vr[0];
+      }
+      fold(sc, vr);
+    }
+    if (live) {
+      TO* op = reinterpret_cast<TO*>(a.O) + row * D + sub * DL;
+      const float inv = 1.f / den;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) store_out<TO>(op + e, ov[e] * inv);
+    }
+  }
+}
+
 // ============================================================ host side
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1177,6 +1515,25 @@ cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
+  dim3 grid((unsigned)((a.n + 16 * kMmaWarps - 1) / (16 * kMmaWarps)),
+            (unsigned)(a.B * a.Hq));
+  const size_t smem = MmaGatherSmem<D>::bytes(a.k);
+  auto k1 = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, 1>
+                     : prefill_gather_mma<D, float, 1>;
+  auto k2 = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, 2>
+                     : prefill_gather_mma<D, float, 2>;
+  auto kern = a.k <= 32 ? k1 : k2;
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  prof_before(s, "prefill_gather");
+  kern<<<grid, kMmaWarps * 32, smem, s>>>(a);
+  prof_after(s);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t prefill_topk_bytes(int B, int n, int Hq, int k) {
@@ -1198,8 +1555,7 @@ cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,
     else e = d == 64 ? launch_select_f32<64>(a, s) : launch_select_f32<128>(a, s);
     if (e != cudaSuccess) return e;
   }
-  if (bf16) e = d == 64 ? launch_gather<__nv_bfloat16, 64>(a, s)
-                        : launch_gather<__nv_bfloat16, 128>(a, s);
+  if (bf16) e = d == 64 ? launch_gather_mma<64>(a, s) : launch_gather_mma<128>(a, s);
   else e = d == 64 ? launch_gather<float, 64>(a, s) : launch_gather<float, 128>(a, s);
   return e;
 }
