@@ -80,8 +80,12 @@ def work_model(w):
                                   "causal score FLOPs: B*H*d*n*(n+1)"),
         "prefill_score_topk_f32": ("alu", flops,
                                    "causal score FLOPs: B*H*d*n*(n+1)"),
-        "prefill_gather": ("hbm", w.B * w.Hq * n * (w.C_max * 4 + w.d * 4),
-                           "idx and O writes: B*H*n*(C_max*4 + d*4)"),
+        "prefill_gather": ("hbm", w.B * w.Hq * n * (w.d * es + w.k * 8 +
+                                                     w.C_max * 4 + 4 + w.d * 4)
+                           + 2 * w.B * w.Hkv * n * w.d * es,
+                           "Q, K, V and Top-k keys read; idx, counts and fp32 O "
+                           "written: B*H*n*(d*e + 8k + 4*C_max + 4 + 4d) + "
+                           "2*B*Hkv*n*d*e"),
     }
 
 
