@@ -517,23 +517,22 @@ decode_merge_attend(DecodeArgs a) {
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (gtid == 0) {
-      s_n = 0;
+      s_n = ncand;
       s_m = 0;
       s_kk = m > 0 ? m : 1;
     }
-    MergeBar::sync();
+    // The lists are copied as they are: empty slots (key 0) sort below every
+    // real key, and the lists hold at least m real keys, so the m-th largest
+    // key is a real one.
     const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
-    for (int e = gtid; e < ncand; e += 256) {
-      const uint64_t key = src[e];
-      if (key != 0ull) cand[atomicAdd(&s_n, 1)] = key;
-    }
+    for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
     MergeBar::sync();
     cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
                                             gtid);
     if (m > 0) {
       for (int e = gtid; e < s_n; e += 256) {
         const uint64_t key = cand[e];
-        if (key >= s_T) {
+        if (key >= s_T && key != 0ull) {
           const uint32_t j = key_index(key);
           const int p = atomicAdd(&s_m, 1);
           if (p < m && j >= 1 && (int64_t)j <= i - Wb) {
