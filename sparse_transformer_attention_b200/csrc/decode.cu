@@ -5,7 +5,7 @@
 //
 // Launch 1, decode_score_topk: grid (chunks, Hkv, B), about two CTAs per SM.
 // One producer thread streams the chunk's contiguous K rows into a ring of
-// 16 KiB shared-memory stages with bulk asynchronous copies (no multicast),
+// 32 KiB shared-memory stages with bulk asynchronous copies (no multicast),
 // so the loads stay deep in flight whatever the compute warps are doing.
 // Eight compute warps read each K row once from shared memory (8 lanes per
 // row, 16-byte reads, conflict-free), score all G = Hq/Hkv q-heads of the
@@ -35,7 +35,11 @@ namespace {
 constexpr int kComputeWarps = 8;
 constexpr int kCompute = kComputeWarps * 32;  // compute threads
 constexpr int kThreads = kCompute + 32;       // + one producer warp
-constexpr int kStageBytes = 16384;
+// Stage size: each stage is waited for and released by every compute warp,
+// so a larger stage spreads that handshake over more keys (32 KiB x 2
+// stages measured 8% faster at 131K and 12% at 1M than 16 KiB x 3).
+constexpr int kStageBytes = 32768;
+constexpr int kTwoCtaStages = 2;  // ring depth when two CTAs share an SM
 constexpr int kMaxStages = 6;  // K staging ring depth (chosen per launch)
 constexpr int kSub = 512;     // keys between candidate-buffer checks
 constexpr int kMinSlack = 256;      // smallest insert room kept after a cut
@@ -219,8 +223,11 @@ struct ScoreCfg {
   static constexpr int ROWB = D * (int)sizeof(T);
   static constexpr int CPL = ROWB / 16 / 8;       // 16-byte pieces per lane
   static constexpr int PPL = CPL * VEC / 2;       // element pairs per lane
-  static constexpr int R = kStageBytes / ROWB;    // K rows per stage
   static constexpr int KPR = 4 * kComputeWarps;   // keys per round
+  // a stage holds a whole number of rounds, about kStageBytes
+  static constexpr int RB = KPR * ROWB;           // bytes per round
+  static constexpr int STAGE = (kStageBytes / RB > 0 ? kStageBytes / RB : 1) * RB;
+  static constexpr int R = STAGE / ROWB;          // K rows per stage
   static constexpr int ROUNDS = R / KPR;
   static constexpr int SUB_ST = kSub / R;         // stages per buffer check
   static_assert(CPL >= 1 && R % KPR == 0 && kSub % R == 0, "tiling");
@@ -253,7 +260,7 @@ decode_score_topk(DecodeArgs a) {
   const int cap = a.cap;  // per-list buffer: k + kSub + slack keys
   const int kStages = a.nstages;
   unsigned char* stages = smem;                                  // ring
-  uint64_t* buf = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * kStageBytes);
+  uint64_t* buf = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * C::STAGE);
   TopkShared<G>* sh = reinterpret_cast<TopkShared<G>*>(buf + (size_t)G * cap);
 
   // Let the merge kernel (launched as a programmatic dependent) start its
@@ -303,7 +310,7 @@ decode_score_topk(DecodeArgs a) {
         const int rows = left < R ? left : R;
         const uint32_t bytes = (uint32_t)rows * C::ROWB;
         sm100::mbar_arrive_expect_tx(&sh->full[s], bytes);
-        sm100::bulk_load(stages + s * kStageBytes, Kg + (size_t)r0 * D, bytes,
+        sm100::bulk_load(stages + s * C::STAGE, Kg + (size_t)r0 * D, bytes,
                          &sh->full[s]);
         issued = t + 1;
         if (++s == kStages) {
@@ -354,7 +361,7 @@ decode_score_topk(DecodeArgs a) {
     const bool ok = __all_sync(
         0xFFFFFFFFu, stage_wait(&sh->full[s], ph, abort_flag, a.status));
     if (ok) {
-      const unsigned char* st = stages + s * kStageBytes;
+      const unsigned char* st = stages + s * C::STAGE;
       const int rbase = c0 + t * R;
 #pragma unroll
       for (int rd = 0; rd < C::ROUNDS; ++rd) {
@@ -611,35 +618,37 @@ decode_merge_attend(DecodeArgs a) {
 }
 
 
-// Shared memory of the score kernel: a K staging ring of 3..kMaxStages
+// Shared memory of the score kernel: a K staging ring of 2..kMaxStages
 // stages and per-list candidate buffers of k + kSub + slack keys.  Prefer
 // two CTAs per SM; spend what is left after the ring on insert slack.
-template <int G>
+template <typename T, int D, int G>
 void score_smem(int k, int* cap, int* nstages, size_t* bytes) {
+  constexpr size_t kStage = ScoreCfg<T, D, G>::STAGE;
   const size_t fixed = sizeof(TopkShared<G>);
   const size_t min_lists = (size_t)G * 8 * (k + kSub + kMinSlack);
   size_t budget = kSmemTwoCtas;
-  if (fixed + min_lists + 3 * (size_t)kStageBytes > budget) budget = kSmemOneCta;
-  // Three stages keep the stream fed (deeper rings measured no faster);
-  // the rest goes to insert slack, which makes list cuts rarer.
+  if (fixed + min_lists + kTwoCtaStages * kStage > budget) budget = kSmemOneCta;
+  // With two CTAs per SM, kTwoCtaStages stages; the rest goes to insert
+  // slack, which makes list cuts rarer (a deeper ring with less slack
+  // measured slower at 131K).
   long st = budget == kSmemTwoCtas
-                ? 3
-                : (long)((budget - fixed - min_lists) / kStageBytes);
+                ? kTwoCtaStages
+                : (long)((budget - fixed - min_lists) / kStage);
   if (st > kMaxStages) st = kMaxStages;
   if (st < 2) st = 2;
-  const size_t rem = budget - fixed - (size_t)st * kStageBytes;
+  const size_t rem = budget - fixed - (size_t)st * kStage;
   long slack = (long)(rem / (8 * G)) - k - kSub;
   if (slack > kMaxSlack) slack = kMaxSlack;
   if (slack < kMinSlack) slack = kMinSlack;
   *cap = k + kSub + (int)slack;
   *nstages = (int)st;
-  *bytes = (size_t)st * kStageBytes + (size_t)G * 8 * (size_t)(*cap) + fixed;
+  *bytes = (size_t)st * kStage + (size_t)G * 8 * (size_t)(*cap) + fixed;
 }
 
 template <typename T, int D, int G>
 cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   size_t smem1;
-  score_smem<G>(a.k, &a.cap, &a.nstages, &smem1);
+  score_smem<T, D, G>(a.k, &a.cap, &a.nstages, &smem1);
   cudaError_t e = cudaSuccess;
   if (a.k > 0) {  // with k = 0 the set is anchor and window only
       auto k1 = decode_score_topk<T, D, G>;
