@@ -394,10 +394,10 @@ decode_score_topk(DecodeArgs a) {
           if (owner && j < c1)
             buf[(size_t)myh * cap + (j - c0)] = make_key(sc, (uint32_t)j);
         } else {
-          // rare once a threshold exists: one warp vote keeps the common
-          // path flat
+          // rare once a threshold exists (a warp vote in front of this
+          // branch measured slower)
           const bool cand = owner && j < c1 && sc >= thr_f;
-          if (__any_sync(0xFFFFFFFFu, cand) && cand) {
+          if (cand) {
             const uint64_t key = make_key(sc, (uint32_t)j);
             if (key > thr) {
               const int pos = atomicAdd(&sh->cnt[myh], 1);
