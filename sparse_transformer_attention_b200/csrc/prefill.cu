@@ -6,17 +6,23 @@
 // Launch 1 (score + select), one CTA per 128-query tile of one (batch, head):
 //   bf16: warp-specialised tcgen05 pipeline.  Warp 0 issues TMA loads of the
 //         Q tile (once) and of 128-key K tiles into a ring of shared-memory
-//         stages; warp 1 issues tcgen05.mma (M=128, N=128, K=16 steps, bf16
-//         in, fp32 out) into one of two TMEM accumulators; warps 2-5 read the
-//         scores back with tcgen05.ld (one thread per query row) and feed the
-//         row's streaming Top-k.  Only key tiles that hold candidates of some
-//         row of the tile are computed (causal tile skipping), and the score
-//         matrix never leaves the SM.
-//   fp32: the same selector fed by an FFMA dot-product loop over 32-key
-//         tiles staged in shared memory (no TF32, so selection stays exact).
+//         stages, twice over (two passes); warp 1 issues tcgen05.mma (M=128,
+//         N=128, K=16 steps, bf16 in, fp32 out) into four TMEM accumulators;
+//         sixteen selector warps read the scores back with tcgen05.ld (thread
+//         = query row x 32-column chunk group).  Pass 1 keeps 128 column-slot
+//         maxima per row, whose k-th largest bounds the row's k-th best score
+//         from below; pass 2 appends every candidate at or above the bound to
+//         the thread's shared-memory segment; the exact Top-k is then cut per
+//         row.  Only key tiles that hold candidates of some row of the tile
+//         are computed, and the score matrix never leaves the SM.  Rows whose
+//         segments overflow go to an exact CUDA-core fallback.
+//   fp32: a per-row heap selector fed by an FFMA dot-product loop over
+//         32-key tiles staged in shared memory (no TF32, so selection stays
+//         exact).
 // Launch 2 (gather + softmax): per row, sort the selected positions, write
 //   C_i (ascending) and |C_i|, and run an fp32 online softmax over
 //   {0} U Top-k U window, re-using the selector's fp32 scores for Top-k.
+//   bf16 runs the window on warp-level MMA, 16 query rows per warp.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
