@@ -1124,7 +1124,7 @@ __device__ __forceinline__ uint32_t bf16_bits_as_f32(const __nv_bfloat16* p) {
 constexpr int kMmaWarps = 4;  // 16 query rows each
 
 // Per warp: the window state (o, max, sum) of its 16 rows, then their Top-k
-// keys as read in step 1.
+// keys as loaded in step 1.
 template <int D>
 struct MmaGatherSmem {
   static constexpr size_t state = (size_t)16 * D * 4 + 2 * 16 * 4;
@@ -1136,7 +1136,8 @@ struct MmaGatherSmem {
 
 // bf16 gather with the window on tensor cores.  A warp owns 16 consecutive
 // query rows of one (batch, head).
-//   1. C_i and |C_i| for each of its rows (whole warp per row).
+//   1. The Top-k keys of its rows into shared memory in one batch of loads,
+//      then C_i and |C_i| for each row (whole warp per row).
 //   2. The window [lo_i, i] of all 16 rows: MMA scores, masked per row, an
 //      online softmax per row over 16-key blocks, and the MMA p * V.  The
 //      state (max, sum, unnormalised o) goes to shared memory.
@@ -1166,7 +1167,28 @@ prefill_gather_mma(PrefillArgs a) {
   const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * n * D;
   const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * n * D;
 
-  // ---- 1: C_i, one row at a time across the warp
+  // ---- 1: the Top-k keys of the warp's rows (16 consecutive rows of one
+  // head: one contiguous run) into shared memory, 16 loads in flight per
+  // lane, then C_i one row at a time across the warp
+  {
+    const int nk = min(16, n - i0) * k;
+    const uint64_t* kg = a.topk + (rowbase + i0) * k;
+#pragma unroll 1
+    for (int e0 = 0; e0 < nk; e0 += 16 * 32) {
+      uint64_t t16[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int e = e0 + u * 32 + lane;
+        t16[u] = e < nk ? __ldg(kg + e) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int e = e0 + u * 32 + lane;
+        if (e < nk) s_key[e] = t16[u];
+      }
+    }
+    __syncwarp();
+  }
 #pragma unroll 1
   for (int rr = 0; rr < 16; ++rr) {
     const int i = i0 + rr;
@@ -1180,8 +1202,7 @@ prefill_gather_mma(PrefillArgs a) {
 #pragma unroll
     for (int t = 0; t < NPL; ++t) {
       const int e = t * 32 + lane;
-      const uint64_t key = e < k ? a.topk[row * k + e] : 0ull;
-      if (e < k) s_key[rr * k + e] = key;
+      const uint64_t key = e < k ? s_key[rr * k + e] : 0ull;
       v[t] = key ? key_index(key) : 0xFFFFFFFFu;
       m += __popc(__ballot_sync(0xFFFFFFFFu, key != 0ull));
     }
@@ -1329,8 +1350,12 @@ prefill_gather_mma(PrefillArgs a) {
 
   // ---- 3: Top-k keys and the anchor, eight lanes per row
   constexpr int DL = D / 8;
-  constexpr int KPC = 4;
+  constexpr int KPC = D == 64 ? 8 : 4;
   const int sub = lane & 7, rq = lane >> 3;
+  // the anchor's K and V rows are the same for all of the warp's rows
+  RawRow<T, DL> k0r, v0r;
+  k0r.load(Kg + sub * DL);
+  v0r.load(Vg + sub * DL);
 #pragma unroll 1
   for (int rg = 0; rg < 4; ++rg) {
     const int r = rg * 4 + rq;
@@ -1392,26 +1417,26 @@ prefill_gather_mma(PrefillArgs a) {
     }
     // the anchor (position 0) when it lies outside the window
     {
-      float sc[KPC];
-      RawRow<T, DL> vr[KPC];
-      RawRow<T, DL> kr;
-      kr.load(Kg + sub * DL);
       float kf[DL];
-      kr.to_f32(kf);
+      k0r.to_f32(kf);
       float d0 = 0.f;
 #pragma unroll
       for (int e = 0; e < DL; ++e) d0 = fmaf(qv[e], kf[e], d0);
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1)
         d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, off);
-      sc[0] = (live && lo > 0) ? d0 * sl2 : -INFINITY;
-      vr[0].load(Vs);
+      if (live && lo > 0) {  // uniform over the row's lanes
+        const float s0 = d0 * sl2;
+        const float mn = fmaxf(mrun, s0);
+        const float f = exp2f(mrun - mn);
+        const float pw = exp2f(s0 - mn);
+        float vf[DL];
+        v0r.to_f32(vf);
+        den = den * f + pw;
 #pragma unroll
-      for (int u = 1; u < KPC; ++u) {
-        sc[u] = -INFINITY;
-        vr[u] = vr[0];
+        for (int e = 0; e < DL; ++e) ov[e] = fmaf(pw, vf[e], ov[e] * f);
+        mrun = mn;
       }
-      fold(sc, vr);
     }
     if (live) {
       TO* op = reinterpret_cast<TO*>(a.O) + row * D + sub * DL;
