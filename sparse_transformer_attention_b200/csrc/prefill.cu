@@ -719,17 +719,23 @@ struct RawRow {
 
 // Exact fallback for rows whose candidate buffer overflowed: one CTA per
 // listed row scores every candidate on CUDA cores (fp32 FMA of the bf16 or
-// fp32 inputs) and keeps the best k keys with the CTA radix select.
+// fp32 inputs).  Scores are taken 2048 keys at a time; a key goes into the
+// buffer only if it reaches the current threshold T (the Top-k so far are
+// exactly the k keys >= T, so a key below T can never be selected), and the
+// CTA radix select runs only when the buffer could not take another chunk,
+// and once at the end.
 constexpr int kFbThreads = 256;
 constexpr int kFbChunk = 2048;
+constexpr int kFbBuf = 2 * kFbChunk;  // buffered keys beyond k
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kFbThreads)
 prefill_overflow_rows(PrefillArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int k = a.k;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);      // [k + chunk]
-  float* q = reinterpret_cast<float*>(keys + k + kFbChunk);  // [D]
+  const int lane = threadIdx.x & 31;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);      // [k + kFbBuf]
+  float* q = reinterpret_cast<float*>(keys + k + kFbBuf);  // [D]
   __shared__ int s_n, s_kk, s_w;
   __shared__ uint64_t s_T;
   __shared__ SelectState<1> st;
@@ -746,37 +752,48 @@ prefill_overflow_rows(PrefillArgs a) {
     const T* Qr = reinterpret_cast<const T*>(a.Q) + (size_t)grow * D;
     const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * a.n * D;
     for (int e = threadIdx.x; e < D; e += kFbThreads) q[e] = Elem<T>::load1(Qr + e);
-    if (threadIdx.x == 0) s_n = 0;
+    if (threadIdx.x == 0) {
+      s_n = 0;
+      s_T = 0ull;  // every real key is above 0
+    }
     __syncthreads();
     for (int c0 = 1; c0 <= hi; c0 += kFbChunk) {
-      for (int jj = threadIdx.x; jj < kFbChunk && c0 + jj <= hi; jj += kFbThreads) {
-        const int j = c0 + jj;
-        // the key row in 16-byte pieces, all loads issued before the FMAs
-        RawRow<T, D> kr;
-        kr.load(Kg + (size_t)j * D);
-        float kf[D];
-        kr.to_f32(kf);
-        float a0 = 0.f, a1 = 0.f;
+      const uint64_t thr = s_T;
+      for (int jj0 = 0; jj0 < kFbChunk; jj0 += kFbThreads) {
+        const int j = c0 + jj0 + (int)threadIdx.x;
+        uint64_t key = 0ull;
+        if (j <= hi) {
+          // the key row in 16-byte pieces, all loads issued before the FMAs
+          RawRow<T, D> kr;
+          kr.load(Kg + (size_t)j * D);
+          float kf[D];
+          kr.to_f32(kf);
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < D; e += 2) {
-          a0 = fmaf(q[e], kf[e], a0);
-          a1 = fmaf(q[e + 1], kf[e + 1], a1);
+          for (int e = 0; e < D; e += 2) {
+            a0 = fmaf(q[e], kf[e], a0);
+            a1 = fmaf(q[e + 1], kf[e + 1], a1);
+          }
+          key = make_key(a0 + a1, (uint32_t)j);
         }
-        keys[s_n + jj] = make_key(a0 + a1, (uint32_t)j);
+        const bool keep = j <= hi && key >= thr;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&s_n, __popc(bal));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        if (keep) keys[base + __popc(bal & ((1u << lane) - 1u))] = key;
       }
       __syncthreads();
-      if (threadIdx.x == 0) {
-        s_n += (hi - c0 + 1 < kFbChunk) ? (hi - c0 + 1) : kFbChunk;
-        s_kk = k;
-      }
-      __syncthreads();
-      cta_select_thresholds<kFbThreads, 1>(keys, 0, &s_n, &s_kk, &s_T, &st,
-                                           threadIdx.x);
-      if (s_n > k) {
+      const bool last = c0 + kFbChunk > hi;
+      if (last ? s_n > k : s_n > k + kFbBuf - kFbChunk) {  // uniform
+        if (threadIdx.x == 0) s_kk = k;
+        __syncthreads();
+        cta_select_thresholds<kFbThreads, 1>(keys, 0, &s_n, &s_kk, &s_T, &st,
+                                             threadIdx.x);
         // keep the keys >= T, packed to the front
         if (threadIdx.x == 0) s_w = 0;
         __syncthreads();
-        uint64_t mine[(kPrefillMaxK + kFbChunk) / kFbThreads + 1];
+        uint64_t mine[(kPrefillMaxK + kFbBuf) / kFbThreads + 1];
         int cntm = 0;
         for (int e = threadIdx.x; e < s_n; e += kFbThreads) mine[cntm++] = keys[e];
         __syncthreads();
@@ -1506,7 +1523,7 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // rows whose segments overflowed (rare on typical inputs): exact fallback
-  const size_t fb_smem = (size_t)(a.k + kFbChunk) * 8 + D * 4;
+  const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
   prof_before(s, "prefill_overflow_rows");
   prefill_overflow_rows<__nv_bfloat16, D><<<148, kFbThreads, fb_smem, s>>>(a);
   prof_after(s);

@@ -90,3 +90,22 @@ def test_prefill_equal_keys_take_the_fallback(d):
     x = workloads.generate(w)
     x["K"][:] = x["K"][:, :, :1, :]
     print(check_prefill(w, x))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_fallback_spans_chunks(d):
+    """K rows at three levels (0.5, 1 and 2 times one row, exact in bf16):
+    rows past position 128 + W tie on more candidates than the row buffer
+    holds and go through the exact fallback, which then scores several
+    2048-key chunks with keys both above and below its running threshold.
+    Rows with q.k_0 > 0 pick the 2x rows, rows with q.k_0 < 0 the 0.5x rows
+    (about half of each); ties go to the lowest indices."""
+    w = workloads.get("prefill_gpt2s_8k").scaled(d=d, n=5000, B=1, Hq=2,
+                                                 Hkv=1, needles=0)
+    x = workloads.generate(w)
+    K = x["K"]
+    K[:] = K[:, :, :1, :]
+    j = np.arange(w.n)
+    c = np.where(j < 3000, 0.5, np.where(j < 4200, 1.0, 2.0))
+    K *= c.astype(K.dtype)[None, None, :, None]
+    print(check_prefill(w, x))
