@@ -49,6 +49,10 @@ def test_workspace_sizes(lib):
     assert ws(True, torch.bfloat16, 1, 131072, 32, 8, 128, 128, 64) > 256
     assert ws(True, torch.bfloat16, 1, 131072, 32, 8, 96, 128, 64) == 0
     assert ws(True, torch.bfloat16, 1, 131072, 30, 8, 128, 128, 64) == 0
+    assert ws(True, torch.bfloat16, 1, 131072, 32, 0, 128, 128, 64) == 0
+    assert ws(False, torch.bfloat16, 1, 0, 32, 8, 128, 128, 64) == 0
+    assert ws(False, torch.bfloat16, 0, 8192, 32, 8, 128, 128, 64) == 0
+    assert ws(False, torch.bfloat16, 1, 8192, 32, 8, 128, 0, 64) == 0
     p = ws(False, torch.bfloat16, 4, 8192, 12, 12, 64, 64, 32)
     assert p >= 256 + 4 * 12 * 8192 * 32 * 8
     assert ws(True, torch.bfloat16, 1, 1 << 20, 32, 8, 128, 256, 128) < (64 << 20)
@@ -86,7 +90,13 @@ def _prefill(lib, **over):
 @pytest.mark.parametrize("call", [_decode, _prefill])
 @pytest.mark.parametrize("over,code", [
     ({"ws": 0}, binding.CA_ERR_WORKSPACE),
+    ({"q": 0}, binding.CA_ERR_INVALID_ARG),
     ({"K": 0}, binding.CA_ERR_INVALID_ARG),
+    ({"idx": 0}, binding.CA_ERR_INVALID_ARG),
+    ({"cnt": 0}, binding.CA_ERR_INVALID_ARG),
+    ({"L": 0}, binding.CA_ERR_INVALID_ARG),
+    ({"Hkv": 0}, binding.CA_ERR_INVALID_ARG),
+    ({"C_max": 0}, binding.CA_ERR_INVALID_ARG),
     ({"O": 0}, binding.CA_ERR_INVALID_ARG),
     ({"B": 0}, binding.CA_ERR_INVALID_ARG),
     ({"k": -1}, binding.CA_ERR_INVALID_ARG),
@@ -103,7 +113,7 @@ def _prefill(lib, **over):
     ({}, binding.CA_ERR_WORKSPACE),  # 16 bytes is never enough
 ])
 def test_invalid_arguments_rejected_before_launch(lib, call, over, code):
-    key_map = {"q": "Q"} if call is _prefill else {}
+    key_map = {"q": "Q", "L": "n"} if call is _prefill else {}
     over = {key_map.get(k, k): v for k, v in over.items()}
     assert call(lib, **over) == code
 
