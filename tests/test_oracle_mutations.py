@@ -34,6 +34,8 @@ MUTATIONS = {
     "value_row_index": ("const float* vj = V + C[r] * (int64_t)d;",
                         "const float* vj = V + r * (int64_t)d;"),
     "normalisation_dropped": ("for (int l = 0; l < d; ++l) o[l] /= den;", ""),
+    "all_candidates_one_short": ("int64_t m = k < ncand ? k : ncand;",
+                                 "int64_t m = k < ncand ? k : ncand - 1;"),
     "score_term_dropped": ("for (int l = 0; l < d; ++l) acc += (double)q[l] * (double)kj[l];",
                            "for (int l = 1; l < d; ++l) acc += (double)q[l] * (double)kj[l];"),
 }
