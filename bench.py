@@ -47,7 +47,10 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD,
                    choices=sorted(workloads.WORKLOADS))
-    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true",
+                   help="skip the CPU leg (oracle timing and parity)")
+    p.add_argument("--no-also", action="store_true",
+                   help="time only --workload, not the rest of the metric")
     return p.parse_args()
 
 
@@ -192,144 +195,127 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- ours
-def run_ours(args, rank, world, local_rank):
+ALSO = ("decode_1m", "prefill_gpt2s_8k", "prefill_adaptive_32k")
+
+
+def config_of(w, world):
+    return {"workload": w.name, "description": w.description,
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            ("L" if w.kind == "decode" else "n"): w.n, "W": w.W, "k": w.k,
+            "adaptive_window": w.adaptive,
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+            "l2": "flushed before every step (256 MiB write), outside the "
+                  "step's events"}
+
+
+class Problem:
+    """Device-resident inputs, outputs and workspace of one workload."""
+
+    def __init__(self, w, dev):
+        import torch
+        import sparse_transformer_attention_b200 as ca
+        self.w, self.dev = w, dev
+        self.x = x = workloads.generate(w)
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tdt)
+        self.Q, self.K, self.V = to(x["Q"]), to(x["K"]), to(x["V"])
+        self.W_i = None if x["W_i"] is None else \
+            torch.from_numpy(x["W_i"]).to(dev)
+        self.decode = w.kind == "decode"
+        if self.decode:
+            self.C_max = min(w.n, 1 + w.W_max + w.k)
+            oshape = (w.B, w.Hq, w.d)
+            ishape = (w.B, w.Hq)
+        else:
+            self.C_max = 1 + w.W_max + w.k
+            oshape = (w.B, w.Hq, w.n, w.d)
+            ishape = (w.B, w.Hq, w.n)
+        self.O = torch.empty(oshape, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(ishape + (self.C_max,), dtype=torch.int32,
+                               device=dev)
+        self.cnt = torch.empty(ishape, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(ca.condensate_attn_workspace_size(
+            self.decode, tdt, w.B, w.n, w.Hq, w.Hkv, w.d, w.W_max, w.k),
+            dtype=torch.uint8, device=dev)
+        self.fn = (ca.condensate_attn_decode if self.decode
+                   else ca.condensate_attn_prefill)
+
+    def step(self, qin=None):
+        w = self.w
+        self.fn(self.Q if qin is None else qin, self.K, self.V, w.W, w.k,
+                W_i=self.W_i, O=self.O, idx=self.idx, idx_count=self.cnt,
+                C_max=self.C_max, workspace=self.ws)
+
+    def status(self):
+        import sparse_transformer_attention_b200 as ca
+        st = ca.condensate_attn_status(self.ws)
+        if st != ca.CA_OK:
+            raise RuntimeError(f"{self.w.name}: device status: "
+                               f"{ca.status_string(st)}")
+
+
+def timed_steps(p, steps, warmup, flush, dist=None, clocks=None):
+    """Device time of each of `steps` steps (CUDA events on the launching
+    stream), after at least `warmup` untimed ones; L2 flushed before every
+    step.  The clock sampler runs from the start of the warm-up (which goes
+    on for at least 0.6 s, so that the samples see the GPU under this load)
+    to the end of the timed steps."""
     import torch
-    import sparse_transformer_attention_b200 as ca
-    from sparse_transformer_attention_b200 import binding
-
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = workloads.get(args.workload)
-    x = workloads.generate(w)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tdt)
-    Q, K, V = to(x["Q"]), to(x["K"]), to(x["V"])
-    W_i = None if x["W_i"] is None else torch.from_numpy(x["W_i"]).to(dev)
-    W_max = w.W_max
-    decode = w.kind == "decode"
-    if decode:
-        C_max = min(w.n, 1 + W_max + w.k)
-        O = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
-        idx = torch.empty((w.B, w.Hq, C_max), dtype=torch.int32, device=dev)
-        cnt = torch.empty((w.B, w.Hq), dtype=torch.int32, device=dev)
-    else:
-        C_max = 1 + W_max + w.k
-        O = torch.empty((w.B, w.Hq, w.n, w.d), dtype=torch.float32, device=dev)
-        idx = torch.empty((w.B, w.Hq, w.n, C_max), dtype=torch.int32,
-                          device=dev)
-        cnt = torch.empty((w.B, w.Hq, w.n), dtype=torch.int32, device=dev)
-    ws = torch.empty(ca.condensate_attn_workspace_size(
-        decode, tdt, w.B, w.n, w.Hq, w.Hkv, w.d, W_max, w.k),
-        dtype=torch.uint8, device=dev)
-    fn = ca.condensate_attn_decode if decode else ca.condensate_attn_prefill
-
-    def step(qin):
-        fn(qin, K, V, w.W, w.k, W_i=W_i, O=O, idx=idx, idx_count=cnt,
-           C_max=C_max, workspace=ws)
-
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
+    if clocks:
+        clocks.start()
+    t_w = time.perf_counter()
+    done = 0
+    while done < warmup or time.perf_counter() - t_w < 0.6:
         flush.zero_()
-        step(Q)
-    st = ca.condensate_attn_status(ws)
-    if st != ca.CA_OK:
-        raise RuntimeError(f"device status: {ca.status_string(st)}")
-    torch.cuda.synchronize()
-
-    uuid = None
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
-    clocks = ClockSampler(uuid)
-    clocks.start()
-    time.sleep(0.3)
-
-    # ---- device-resident timed region
+        p.step()
+        done += 1
+        if done % 8 == 0:
+            torch.cuda.synchronize()
+    p.status()
     evs = [(torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    for s in range(args.steps):
+    for s in range(steps):
         flush.zero_()  # L2 flush, outside the step's events
         evs[s][0].record()
-        step(Q)
+        p.step()
         evs[s][1].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
+    clk = clocks.stop() if clocks else None
     if dist:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    # Per-kernel device times come from a separate pass: the library's event
-    # records between its launches would otherwise serialise the dependent
-    # launch of the second kernel inside the timed steps.
-    binding.profile_start(8 * args.steps + 16)
-    for s in range(args.steps):
+    return [a.elapsed_time(b) for a, b in evs], wall, clk
+
+
+def kernel_times(p, steps, flush):
+    """Per-launch device times from the library's own events, in a separate
+    pass: event records between the library's launches would otherwise
+    serialise the dependent launch of the second kernel inside the timed
+    steps."""
+    import torch
+    from sparse_transformer_attention_b200 import binding
+    binding.profile_start(16 * steps + 16)
+    for _ in range(steps):
         flush.zero_()
-        step(Q)
+        p.step()
     torch.cuda.synchronize()
-    prof = binding.profile_stop(8 * args.steps + 16)
-
-    # ---- end to end through the public API with host buffers
-    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-    if decode:
-        q_host = pin(Q)
-        q_host.copy_(Q.cpu())
-        q_dev = torch.empty_like(Q)
-        h2d = q_host.numel() * q_host.element_size()
-    else:
-        # prefill consumes Q, K and V of the step
-        hosts = [pin(t) for t in (Q, K, V)]
-        for h_, t_ in zip(hosts, (Q, K, V)):
-            h_.copy_(t_.cpu())
-        h2d = sum(h_.numel() * h_.element_size() for h_ in hosts)
-    outs = [pin(O), pin(idx), pin(cnt)]
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    e2e_ev = [(torch.cuda.Event(enable_timing=True),
-               torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for s in range(args.steps):
-        flush.zero_()
-        e2e_ev[s][0].record()
-        if decode:
-            q_dev.copy_(q_host, non_blocking=True)
-            step(q_dev)
-        else:
-            Q.copy_(hosts[0], non_blocking=True)
-            K.copy_(hosts[1], non_blocking=True)
-            V.copy_(hosts[2], non_blocking=True)
-            step(Q)
-        for o_h, o_d in zip(outs, (O, idx, cnt)):
-            o_h.copy_(o_d, non_blocking=True)
-        e2e_ev[s][1].record()
-    torch.cuda.synchronize()
-    e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
-    clk = clocks.stop()
-    st = ca.condensate_attn_status(ws)
-    if st != ca.CA_OK:
-        raise RuntimeError(f"device status: {ca.status_string(st)}")
-
-    ms = statistics.mean(step_ms)
-    e2e_mean = statistics.mean(e2e_ms)
-    if dist:
-        ms, e2e_mean = max_over_ranks([ms, e2e_mean], device=dev)
-
-    # per-kernel device times
+    prof = binding.profile_stop(16 * steps + 16)
     per = {}
     for name, t in prof:
         per.setdefault(name, []).append(t)
-    kern_avg = {k_: statistics.mean(v) for k_, v in per.items()}
-    launches = len(prof)  # library kernels launched per timed pass
-    pk = peaks()
+    return per, len(prof)
+
+
+def roofline_of(w, per, pk, sm_max_mhz):
+    """Roofline of the dominant kernel among those with a work model (the
+    exact fallback for overflowing prefill rows has none: its work depends
+    on the rows)."""
     model = work_model(w)
-    # the dominant kernel among those with a work model (the exact fallback
-    # for overflowing prefill rows has none: its work depends on the rows)
+    kern_avg = {k_: statistics.mean(v) for k_, v in per.items()}
     dom = max((k_ for k_ in kern_avg if k_ in model),
               key=lambda k_: sum(per[k_]))
     bound, work, what = model[dom]
@@ -343,45 +329,147 @@ def run_ours(args, rank, world, local_rank):
     else:
         achieved = work / t_dom / 1e12
         # fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock
-        peak = 148 * 128 * 2 * (clk["sm_max_mhz"] or 1965.0) * 1e6 / 1e12
+        peak = 148 * 128 * 2 * (sm_max_mhz or 1965.0) * 1e6 / 1e12
         unit = "TFLOP/s"
-    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+    return {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
             "unit": unit, "frac": achieved / peak,
             "peak_source": pk["source"] + (" burst" if bound != "alu" else
                                            " derived"),
             "work_per_launch": work, "work_definition": what,
             "avg_launch_ms": kern_avg[dom],
-            "traffic": traffic_for(dom, w.name)}
-    units = step_units(w) * world
+            "traffic": traffic_for(dom, w.name)}, kern_avg
+
+
+def step_roofline_of(w, ms, pk):
+    model = work_model(w)
+    if w.kind == "decode":
+        # whole-step HBM roofline: K scored + K/V rows of C_i gathered
+        b = model["decode_score_topk"][1] + model["decode_merge_attend"][1]
+        return {"bytes": b, "achieved_gbs": b / (ms * 1e-3) / 1e9,
+                "frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    f = model["prefill_score_topk_tc"][1]
+    t = f / (ms * 1e-3) / 1e12
+    return {"flops": f, "achieved_tflops": t, "frac": t / pk["bf16_tflops"]}
+
+
+def e2e_of(p, steps, flush):
+    """The same metric through the public call with host buffers: every step
+    copies its inputs from pinned host memory and reads the outputs back."""
+    import torch
+    w = p.w
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    if p.decode:
+        q_host = pin(p.Q)
+        q_host.copy_(p.Q.cpu())
+        q_dev = torch.empty_like(p.Q)
+        h2d = q_host.numel() * q_host.element_size()
+    else:
+        # prefill consumes Q, K and V of the step
+        hosts = [pin(t) for t in (p.Q, p.K, p.V)]
+        for h_, t_ in zip(hosts, (p.Q, p.K, p.V)):
+            h_.copy_(t_.cpu())
+        h2d = sum(h_.numel() * h_.element_size() for h_ in hosts)
+    outs = [pin(p.O), pin(p.idx), pin(p.cnt)]
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.zero_()
+        evs[s][0].record()
+        if p.decode:
+            q_dev.copy_(q_host, non_blocking=True)
+            p.step(q_dev)
+        else:
+            p.Q.copy_(hosts[0], non_blocking=True)
+            p.K.copy_(hosts[1], non_blocking=True)
+            p.V.copy_(hosts[2], non_blocking=True)
+            p.step()
+        for o_h, o_d in zip(outs, (p.O, p.idx, p.cnt)):
+            o_h.copy_(o_d, non_blocking=True)
+        evs[s][1].record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return ms, h2d, d2h
+
+
+def measure(w, dev, steps, warmup, flush, pk, uuid, dist=None, world=1):
+    """Timed steps, clocks, per-kernel times and rooflines of one workload."""
+    p = Problem(w, dev)
+    step_ms, wall, clk = timed_steps(p, steps, warmup, flush, dist,
+                                     ClockSampler(uuid))
+    per, launches = kernel_times(p, steps, flush)
+    p.status()
+    ms = statistics.mean(step_ms)
+    roof, kern_avg = roofline_of(w, per, pk, clk.get("sm_max_mhz"))
+    rec = {"ms_per_step": ms, "tokens_per_s": job_rate(step_units(w), world, ms),
+           "roofline": roof, "step_roofline": step_roofline_of(w, ms, pk),
+           "kernels_avg_ms": kern_avg,
+           "kernel_launches_per_step": launches / steps,
+           "clocks": clk, "config": config_of(w, world)}
+    return p, rec, step_ms, launches, wall
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.get(args.workload)
+    pk = peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+
+    p, rec, step_ms, launches, wall = measure(
+        w, dev, args.steps, args.warmup, flush, pk, uuid, dist, world)
+    e2e_ms, h2d, d2h = e2e_of(p, args.steps, flush)
+    p.status()
+    ms = rec["ms_per_step"]
+    if dist:
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
+    # the rest of the metric, one workload at a time (one GPU only: every
+    # rank of a replicated run would otherwise repeat them)
+    also = {}
+    if world == 1 and not args.no_also:
+        headline = p
+        for name in ALSO:
+            if name == w.name:
+                continue
+            q, r, *_ = measure(workloads.get(name), dev, args.steps,
+                               args.warmup, flush, pk, uuid)
+            if rank == 0 and not args.no_cpu_baseline:
+                r["parity"] = parity_of(q, sample_rows=2000)
+            also[name] = r
+            del q
+            torch.cuda.empty_cache()
+        p = headline
+
+    decode = w.kind == "decode"
     rate = job_rate(step_units(w), world, ms)
     if decode:
         value, unit_v, hib = ms, "ms", False
-        # whole-step HBM roofline: K scored + K/V rows of C_i gathered
-        step_bytes = (model["decode_score_topk"][1]
-                      + model["decode_merge_attend"][1])
-        step_roof = {"bytes": step_bytes,
-                     "achieved_gbs": step_bytes / (ms * 1e-3) / 1e9,
-                     "frac": step_bytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-        e2e_val, e2e_unit = e2e_mean, "ms"
+        e2e_val, e2e_unit = e2e_ms, "ms"
     else:
         value, unit_v, hib = rate, "tokens/s", True
-        step_roof = {"flops": work, "achieved_tflops":
-                     model["prefill_score_topk_tc"][1] / (ms * 1e-3) / 1e12}
-        e2e_val, e2e_unit = job_rate(step_units(w), world, e2e_mean), "tokens/s"
+        e2e_val, e2e_unit = job_rate(step_units(w), world, e2e_ms), "tokens/s"
     out = {
         "metric": METRIC, "value": value, "unit": unit_v, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": hib, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded; see workloads/)",
-        "config": {"workload": w.name, "description": w.description,
-                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   ("L" if decode else "n"): w.n, "W": w.W, "k": w.k,
-                   "adaptive_window": w.adaptive,
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "l2": "flushed before every step (256 MiB write), "
-                         "outside the step's events"},
-        "roofline": roof, "step_roofline": step_roof,
-        "kernels_avg_ms": kern_avg,
+        "config": config_of(w, world),
+        "roofline": rec["roofline"],
+        "step_roofline": step_roofline_of(w, ms, pk),
+        "kernels_avg_ms": rec["kernels_avg_ms"],
         "tokens_per_s": rate,
         "e2e": {"value": e2e_val, "unit": e2e_unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -389,15 +477,79 @@ def run_ours(args, rank, world, local_rank):
                          "O/idx/count D2H" if decode else
                          "Q/K/V H2D, call, O/idx/count D2H")},
         "gpu_launches": launches,
-        "clocks": clk,
+        "clocks": rec["clocks"],
         "wall_s_timed_region": wall,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        out["cpu_baseline"] = cpu_baseline(w, x, budget_s=15.0)
+        # the CPU leg: the oracle timed on a bounded sample, and the parity
+        # of this run's last step against it
+        out["cpu_baseline"] = cpu_baseline(w, p.x, budget_s=15.0)
+        out["parity"] = parity_of(p, sample_rows=4000)
+    if also:
+        out["also"] = also
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     return out
+
+
+def parity_of(p, sample_rows):
+    """Rows of the last step compared with the oracle: index sets identical
+    outside near-ties (swaps inside the rounding bound), outputs within the
+    tolerance.  Decode: every (batch, q-head); prefill: a seeded sample of
+    rows plus every row the selector sent to its exact fallback."""
+    import oracle
+    from oracle.parity import check_rows
+    w, x = p.w, p.x
+    tol = 1e-2 if w.dtype == "bf16" else 1e-5
+    G = w.Hq // w.Hkv
+    try:
+        if p.decode:
+            ref = oracle.decode(x["Q"], x["K"], x["V"], w.W, w.k,
+                                W_i=x["W_i"], C_max=p.C_max, with_full=False)
+            rows = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+            win = [int(x["W_i"][b]) if x["W_i"] is not None else w.W
+                   for (b, h) in rows]
+            r = check_rows(
+                ref, p.idx.cpu().numpy(), p.cnt.cpu().numpy(),
+                p.O.float().cpu().numpy(),
+                q_rows=[x["Q"][b, h] for (b, h) in rows],
+                kv_rows=lambda i: x["K"][rows[i][0], rows[i][1] // G],
+                v_rows=lambda i: x["V"][rows[i][0], rows[i][1] // G],
+                pos=[w.n - 1] * len(rows), win=win, tol=tol)
+            r["what"] = "every (batch, q-head) row"
+            return r
+        import torch
+        rng = np.random.default_rng(0)
+        sel = np.stack([rng.integers(w.B, size=sample_rows),
+                        rng.integers(w.Hq, size=sample_rows),
+                        rng.integers(w.n, size=sample_rows)], 1)
+        R = w.B * w.Hq * w.n
+        nfb = int(p.ws[16:20].cpu().numpy().view(np.uint32)[0])
+        off = 256 + (R * max(w.k, 1) * 8 + 255) // 256 * 256
+        fb = p.ws[off:off + 4 * nfb].cpu().numpy().view(np.uint32)
+        bh, i_ = np.divmod(fb.astype(np.int64), w.n)
+        fb = np.stack([bh // w.Hq, bh % w.Hq, i_], 1)
+        sel = np.unique(np.concatenate([sel, fb.reshape(-1, 3)]), axis=0)
+        ti = torch.from_numpy(sel).to(p.dev)
+        g_idx = p.idx[ti[:, 0], ti[:, 1], ti[:, 2]].cpu().numpy()
+        g_cnt = p.cnt[ti[:, 0], ti[:, 1], ti[:, 2]].cpu().numpy()
+        g_o = p.O[ti[:, 0], ti[:, 1], ti[:, 2]].float().cpu().numpy()
+        ref = oracle.prefill(x["Q"], x["K"], x["V"], w.W, w.k, W_i=x["W_i"],
+                             sel=sel, C_max=p.C_max, with_full=False)
+        win = [int(x["W_i"][b, i]) if x["W_i"] is not None else w.W
+               for (b, h, i) in sel]
+        r = check_rows(
+            ref, g_idx, g_cnt, g_o,
+            q_rows=[x["Q"][b, h, i] for (b, h, i) in sel],
+            kv_rows=lambda i: x["K"][sel[i][0], sel[i][1] // G],
+            v_rows=lambda i: x["V"][sel[i][0], sel[i][1] // G],
+            pos=sel[:, 2], win=win, tol=tol)
+        r["what"] = (f"{sample_rows} seeded sample rows + {nfb} exact-"
+                     f"fallback rows")
+        return r
+    except AssertionError as e:
+        return {"failed": str(e)[:300]}
 
 
 # ----------------------------------------------------------------- oracle
@@ -458,7 +610,7 @@ def run_reference(args):
         "higher_is_better": not decode, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; see workloads/)",
-        "config": {"workload": w.name, "description": w.description},
+        "config": config_of(w, args.gpus),
         "cpu_baseline": cb,
         "e2e": {"value": v, "unit": cb["unit"], "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -33,10 +33,20 @@
  * Scores and the softmax are accumulated in fp32; selection uses the
  * unscaled fp32 dot product with the tie rule above.
  *
- * Ownership: every pointer is a device pointer owned by the caller; the
- * library allocates nothing and keeps no global mutable state.  `stream` is a
- * cudaStream_t (NULL = legacy default stream).  Calls are asynchronous; the
- * returned status covers argument checks and launch errors only.
+ * Ownership: every pointer is a device pointer owned by the caller, and no
+ * entry point allocates device memory.  `stream` is a cudaStream_t (NULL =
+ * legacy default stream).  Calls are asynchronous; the returned status
+ * covers argument checks and launch errors only.
+ *
+ * Process-wide state (everything else is per call): a per-device cache of
+ * kernel attributes and of the SM count (filled on first use, behind a
+ * mutex); the profiling switch (condensate_attn_profile_start/stop) and the
+ * failure-path test hook (condensate_attn_test_stall), both for benchmarks
+ * and tests, not for use while other threads call the library; and the
+ * built-in buffer of condensate_attn_decode_noalloc with its per-device
+ * address cache.  The decode chunking follows the current device's SM count,
+ * so query condensate_attn_workspace_size with the device current that the
+ * call will run on.
  *
  * Errors: arguments are validated before anything is launched (null
  * pointers, sizes, d, group size, 16-byte alignment, C_max >= 1+W+k for the
@@ -70,7 +80,9 @@ typedef enum {
   CA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required         */
   CA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed            */
   CA_ERR_TIMEOUT = 6,     /* a bounded device wait gave up (status query)    */
-  CA_ERR_DEVICE_ARG = 7   /* W_i out of range or set overflowing C_max      */
+  CA_ERR_DEVICE_ARG = 7,  /* W_i out of range or set overflowing C_max      */
+  CA_ERR_INTERNAL = 8     /* an internal check failed on the device: the
+                             results of that call are invalid (a bug)      */
 } ca_status;
 
 typedef enum { CA_F32 = 0, CA_BF16 = 1 } ca_dtype;
@@ -125,10 +137,12 @@ CA_API ca_status condensate_attn_decode(const void* q, const void* K, const void
  * decode workspace (condensate_attn_workspace_size) exceeds 4 MiB are
  * rejected with CA_ERR_WORKSPACE before any launch.  Allocates nothing.  The
  * first call on a device looks up the buffer's device address; make it
- * before any stream capture.  All calls on a device share the buffer: calls
- * that overlap on the GPU race and must be serialised by the caller.
- * Device-side flags (W_i below 1, C_max overflow) land in the shared buffer
- * and are not reported by this entry point.
+ * before any stream capture.  That address is cached for the life of the
+ * device's primary context: do not call this entry point again after
+ * cudaDeviceReset.  All calls on a device share the buffer: calls that
+ * overlap on the GPU race and must be serialised by the caller.  Flags the
+ * kernels raise on the device land in the shared buffer's status word; read
+ * them with condensate_attn_decode_noalloc_status.
  */
 CA_API ca_status condensate_attn_decode_noalloc(
     const void* q, const void* K, const void* V, ca_dtype dtype, int B, int L,
@@ -137,11 +151,40 @@ CA_API ca_status condensate_attn_decode_noalloc(
     void* stream);
 
 /*
+ * Status of the last condensate_attn_decode_noalloc call(s) on the current
+ * device: waits for `stream`, then reads and clears the status word of the
+ * built-in buffer, with the codes of condensate_attn_status.  Allocates
+ * nothing.  The paper has no counterpart to this entry point.
+ */
+CA_API ca_status condensate_attn_decode_noalloc_status(void* stream);
+
+/*
  * Waits for `stream`, then reads and clears the device status word of
- * `workspace`: CA_OK, CA_ERR_DEVICE_ARG or CA_ERR_TIMEOUT (CA_ERR_CUDA if
- * the wait or copy itself failed).
+ * `workspace`.  The kernels raise four flags there:
+ *   W_i below 1                      -> CA_ERR_DEVICE_ARG (the row is run
+ *                                       with a window of 1)
+ *   |C_i| larger than C_max          -> CA_ERR_DEVICE_ARG (idx holds the
+ *                                       first C_max entries, idx_count the
+ *                                       true size)
+ *   a bounded device wait ran out    -> CA_ERR_TIMEOUT (outputs invalid)
+ *   an internal check failed         -> CA_ERR_INTERNAL (outputs invalid)
+ * The time-out outranks the argument flags, which outrank the internal one.
+ * CA_OK when no flag is set; CA_ERR_CUDA if the wait or copy itself failed.
  */
 CA_API ca_status condensate_attn_status(void* workspace, void* stream);
+
+/*
+ * Failure-path test hook, not for production use.  With limit_ns > 0 every
+ * later prefill or decode call makes one pipeline consumer of its score
+ * kernel wait, for at most limit_ns, on a barrier that nothing signals: the
+ * wait runs out, the kernel raises the time-out flag, every other wait of
+ * the CTA gives up at once, and the kernel leaves through its normal path
+ * (copies and tensor-core operations it issued are drained first), so the
+ * CUDA context stays usable and condensate_attn_status reports
+ * CA_ERR_TIMEOUT.  0 turns the hook off.  Process-wide switch; limit_ns
+ * above 60 s is CA_ERR_INVALID_ARG.
+ */
+CA_API ca_status condensate_attn_test_stall(unsigned long long limit_ns);
 
 /* Static, human-readable name of a status code. */
 CA_API const char* condensate_attn_status_string(ca_status s);

@@ -24,6 +24,7 @@ CA_ERR_WORKSPACE = 4
 CA_ERR_CUDA = 5
 CA_ERR_TIMEOUT = 6
 CA_ERR_DEVICE_ARG = 7
+CA_ERR_INTERNAL = 8
 
 CA_F32 = 0
 CA_BF16 = 1
@@ -43,7 +44,9 @@ SIGNATURES = {
     "condensate_attn_decode_noalloc":
         (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
               _I, _P]),
+    "condensate_attn_decode_noalloc_status": (_I, [_P]),
     "condensate_attn_status": (_I, [_P, _P]),
+    "condensate_attn_test_stall": (_I, [ctypes.c_ulonglong]),
     "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
     "condensate_attn_version": (_I, []),
     "condensate_attn_profile_start": (_I, [_I]),
@@ -204,6 +207,12 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
 def condensate_attn_status(workspace: torch.Tensor, stream=None) -> int:
     """Wait for the stream and return (and clear) the device status code."""
     return int(load().condensate_attn_status(_ptr(workspace), _stream(stream)))
+
+
+def test_stall(limit_ns: int) -> None:
+    """Failure-path test hook (see the header): 0 turns it off."""
+    _check(load().condensate_attn_test_stall(int(limit_ns)),
+           "condensate_attn_test_stall")
 
 
 def profile_start(capacity: int = 4096) -> None:

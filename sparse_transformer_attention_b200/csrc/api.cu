@@ -3,12 +3,17 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/condensate_attn.h"
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
 
 namespace {
+
+// Failure-path test hook (condensate_attn_test_stall): 0 = off.
+std::atomic<unsigned long long> g_stall_ns{0};
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -47,6 +52,7 @@ const char* condensate_attn_status_string(ca_status s) {
     case CA_ERR_CUDA: return "CUDA error";
     case CA_ERR_TIMEOUT: return "device wait timed out";
     case CA_ERR_DEVICE_ARG: return "device-side argument out of range";
+    case CA_ERR_INTERNAL: return "internal consistency check failed on the device";
   }
   return "unknown status";
 }
@@ -113,6 +119,8 @@ ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
   a.kpow2 = next_pow2(k > 1 ? k : 2);
   a.status = (uint32_t*)workspace;
   a.cand = (uint64_t*)((char*)workspace + ca::kStatusBytes);
+  a.wait_ns = ca::kPipelineWaitNs;
+  a.stall_ns = g_stall_ns.load();
   cudaError_t e = ca::decode_launch(a, dtype == CA_BF16, d, s);
   return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
 }
@@ -145,6 +153,8 @@ ca_status condensate_attn_prefill(const void* Q, const void* K, const void* V,
   a.ovf_count = (uint32_t*)workspace + 4;  // inside the cleared status area
   a.topk = (uint64_t*)((char*)workspace + ca::kStatusBytes);
   a.ovf_rows = (uint32_t*)((char*)a.topk + ca::prefill_topk_bytes(B, n, Hq, k));
+  a.wait_ns = ca::kPipelineWaitNs;
+  a.stall_ns = g_stall_ns.load();
   cudaError_t e = ca::prefill_launch(a, dtype == CA_BF16, d, s);
   if (e == cudaErrorNotSupported) return CA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
@@ -161,7 +171,13 @@ ca_status condensate_attn_status(void* workspace, void* stream) {
     return CA_ERR_CUDA;
   if (word & ca::kErrTimeout) return CA_ERR_TIMEOUT;
   if (word & (ca::kErrWindow | ca::kErrCmax)) return CA_ERR_DEVICE_ARG;
-  if (word & ca::kErrInternal) return CA_ERR_CUDA;
+  if (word & ca::kErrInternal) return CA_ERR_INTERNAL;
+  return CA_OK;
+}
+
+ca_status condensate_attn_test_stall(unsigned long long limit_ns) {
+  if (limit_ns > 60ull * 1000000000ull) return CA_ERR_INVALID_ARG;
+  g_stall_ns.store(limit_ns);
   return CA_OK;
 }
 

@@ -15,6 +15,13 @@ constexpr uint32_t kErrInternal = 8u;  // internal capacity check failed
 
 constexpr int kStatusBytes = 256;      // status area at the workspace start
 
+// Limits of the bounded waits.  A pipeline wait (a consumer waiting for its
+// producer) gives up after kPipelineWaitNs and aborts the CTA; a drain wait
+// (a thread waiting for copies or MMAs it issued itself, before exit) is
+// always given kDrainWaitNs.
+constexpr uint64_t kPipelineWaitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kDrainWaitNs = 2000000000ull;     // 2 s
+
 __device__ __forceinline__ void raise_flag(uint32_t* status, uint32_t bit) {
   atomicOr(status, bit);
 }

@@ -23,6 +23,7 @@
 // with their keys; the two partial softmax states are then combined.
 #include "common.cuh"
 #include "decode.cuh"
+#include "launch.cuh"
 #include "profile.cuh"
 #include "select.cuh"
 #include "sm100.cuh"
@@ -47,7 +48,6 @@ constexpr int kMaxSlack = 2048;     // largest useful insert room
 constexpr size_t kSmemTwoCtas = 108 * 1024;   // two CTAs per SM, with margin
 constexpr size_t kSmemOneCta = 227 * 1024;
 constexpr int kMergeThreads = 512;
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per bounded wait
 using ComputeBar = GroupBarrier<1, kCompute>;
 using MergeBar = GroupBarrier<1, 256>;
 
@@ -98,29 +98,12 @@ __device__ __forceinline__ bool reduce_owner(int l8) {
 template <int G>
 struct TopkShared {
   uint64_t full[kMaxStages], empty[kMaxStages];
+  uint64_t never;  // failure-path test hook: a barrier nothing signals
   uint64_t thr[G];
   int cnt[G];
   int abort;
   uint32_t hist[G][256];  // one radix histogram per list (per cutting warp)
 };
-
-// Bounded wait on a stage barrier; a time-out raises the CTA's abort flag
-// (and the status bit) so that every other wait returns at once.
-__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity,
-                                           volatile int* abort_flag,
-                                           uint32_t* status) {
-  if (sm100::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = sm100::globaltimer_ns();
-  while (true) {
-    if (sm100::mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (sm100::globaltimer_ns() - t0 > kWaitNs) {
-      *abort_flag = 1;
-      raise_flag(status, kErrTimeout);
-      return false;
-    }
-  }
-}
 
 // One warp cuts the list lst[0..n) of unique keys down to its best kk keys
 // (n > kk >= 1), in place and in no particular order, and returns the
@@ -285,6 +268,7 @@ decode_score_topk(DecodeArgs a) {
       sm100::mbar_init(&sh->full[s], 1);
       sm100::mbar_init(&sh->empty[s], kComputeWarps);
     }
+    sm100::mbar_init(&sh->never, 1);
     for (int h = 0; h < G; ++h) {
       sh->cnt[h] = 0;
       sh->thr[h] = 0ull;
@@ -303,7 +287,8 @@ decode_score_topk(DecodeArgs a) {
       uint32_t ph = 0;  // parity of the ring pass of stage s
       for (int t = 0; t < nst; ++t) {
         if (t >= kStages &&
-            !stage_wait(&sh->empty[s], ph ^ 1, abort_flag, a.status))
+            !sm100::wait_or_abort(&sh->empty[s], ph ^ 1, abort_flag, a.status,
+                                  a.wait_ns))
           break;
         const int r0 = c0 + t * R;
         const int left = nrows - t * R;
@@ -320,12 +305,20 @@ decode_score_topk(DecodeArgs a) {
       }
       // every copy this thread started must land before the CTA exits
       for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
-        sm100::mbar_wait(&sh->full[t % kStages], (t / kStages) & 1, kWaitNs);
+        if (!sm100::mbar_wait(&sh->full[t % kStages], (t / kStages) & 1,
+                              kDrainWaitNs))
+          raise_flag(a.status, kErrTimeout);
     }
     return;
   }
 
   // -------------------------------------------------- compute warps
+  if (a.stall_ns && warp == 0) {
+    // Failure-path test hook: wait on a barrier that nothing signals, so the
+    // wait runs out, raises the time-out flag and aborts every wait of the
+    // CTA; the kernel then leaves through its normal path.
+    sm100::wait_or_abort(&sh->never, 0, abort_flag, a.status, a.stall_ns);
+  }
   const int l8 = lane & 7, ks = lane >> 3;
   float2 q2[G][PPL];
 #pragma unroll
@@ -359,7 +352,8 @@ decode_score_topk(DecodeArgs a) {
       thr_f = thr ? key_score(thr) : -INFINITY;
     }
     const bool ok = __all_sync(
-        0xFFFFFFFFu, stage_wait(&sh->full[s], ph, abort_flag, a.status));
+        0xFFFFFFFFu, sm100::wait_or_abort(&sh->full[s], ph, abort_flag,
+                                          a.status, a.wait_ns));
     if (ok) {
       const unsigned char* st = stages + s * C::STAGE;
       const int rbase = c0 + t * R;
@@ -652,12 +646,8 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
   if (a.k > 0) {  // with k = 0 the set is anchor and window only
       auto k1 = decode_score_topk<T, D, G>;
-    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem1);
-    if (e != cudaSuccess) return e;
-    // ask for the largest shared-memory carve-out so two CTAs fit per SM
-    e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
+    // the largest shared-memory carve-out, so that two CTAs fit per SM
+    e = ensure_smem(k1, smem1, true);
     if (e != cudaSuccess) return e;
     dim3 grid1(a.nchunks, a.Hkv, a.B);
     prof_before(stream, "decode_score_topk");
@@ -671,8 +661,7 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   dim3 grid2(a.Hq, a.B);
   auto k2 = a.o_bf16 ? decode_merge_attend<T, D, __nv_bfloat16>
                      : decode_merge_attend<T, D, float>;
-  e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem2);
+  e = ensure_smem(k2, smem2);
   if (e != cudaSuccess) return e;
   // Programmatic dependent launch: the merge grid may start while the score
   // grid drains; it waits (griddepcontrol.wait) before reading the lists.
@@ -707,10 +696,11 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 int decode_chunks(int B, int L, int Hkv, int k) {
-  // About two CTAs per SM of a 148-SM part, each chunk a multiple of 64 keys,
-  // and at most 8192 merged candidates per q-head.
+  // About two CTAs per SM of the current device, each chunk a multiple of
+  // 64 keys, and at most 8192 merged candidates per q-head.
   const int units = B * Hkv;
-  int per = (kDecodeTargetCtas + units - 1) / units;
+  const int target = kDecodeCtasPerSm * sm_count();
+  int per = (target + units - 1) / units;
   int cap_merge = kDecodeMaxMerge / (k > 0 ? k : 1);
   if (per > cap_merge) per = cap_merge;
   int max_by_len = (L + 255) / 256;

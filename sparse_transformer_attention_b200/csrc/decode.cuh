@@ -6,8 +6,9 @@
 
 namespace ca {
 
-// About two CTAs per SM on a 148-SM B200 for the K-streaming pass.
-constexpr int kDecodeTargetCtas = 296;
+// CTAs per SM of the K-streaming pass (the grid is this times the SM count
+// of the current device, split over batch x kv-heads x chunks).
+constexpr int kDecodeCtasPerSm = 2;
 // Largest Top-k of the decode path (the per-head candidate buffers of the
 // score pass must fit in shared memory next to the K staging ring).
 constexpr int kDecodeMaxK = 1024;
@@ -31,6 +32,8 @@ struct DecodeArgs {
   int nstages;          // K staging ring depth of the score kernel
   uint64_t* cand;       // [B, Hq, nchunks, k] chunk-best keys (workspace)
   uint32_t* status;   // device status word (workspace)
+  uint64_t wait_ns;   // limit of each pipeline wait (kPipelineWaitNs)
+  uint64_t stall_ns;  // failure-path test hook (0: off)
 };
 
 int decode_chunks(int B, int L, int Hkv, int k);

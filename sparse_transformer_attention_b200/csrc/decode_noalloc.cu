@@ -17,7 +17,12 @@
 //
 // All calls on a device share the one buffer and it keeps the previous
 // call's contents: the status word at its start is cleared by every call,
-// and the candidate lists are fully rewritten before they are read.  Calls
+// and the candidate lists are fully rewritten before they are read.  The
+// flags a call raises on the device (a bad W_i, an overflowing C_max, a
+// bounded wait that ran out, a failed internal check) are read and cleared
+// by condensate_attn_decode_noalloc_status.  The cached address is valid for
+// the life of the device's primary context: after cudaDeviceReset the
+// process must not call these entry points again.  Calls
 // that overlap on the GPU (on different streams, or from several host
 // threads) race on the buffer and must be serialised by the caller.  The
 // call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
@@ -71,4 +76,13 @@ extern "C" ca_status condensate_attn_decode_noalloc(
   return condensate_attn_decode(q, K, V, dtype, B, L, Hq, Hkv, d, W, k, W_i,
                                 O, o_dtype, idx, idx_count, C_max, scratch,
                                 kScratchBytes, stream);
+}
+
+// The device status word of the built-in buffer lives at its start, like a
+// workspace's; reading it reuses the cached address and allocates nothing.
+extern "C" ca_status condensate_attn_decode_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  ca_status st = scratch_address(&scratch);
+  if (st != CA_OK) return st;
+  return condensate_attn_status(scratch, stream);
 }

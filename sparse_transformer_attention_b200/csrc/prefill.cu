@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "prefill.cuh"
 #include "profile.cuh"
 #include "row_topk.cuh"
@@ -36,8 +37,6 @@
 namespace ca {
 
 namespace {
-
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
 
 // ------------------------------------------------------------ shared prologue
 // Window and last candidate position of each row of the tile; returns the
@@ -115,6 +114,7 @@ struct TcLayout {
 
 struct TcShared {
   uint64_t kfull[4], kempty[4], qfull, tfull[kTmemBufs], tempty[kTmemBufs];
+  uint64_t never;  // failure-path test hook: a barrier nothing signals
   uint32_t tmem;
   int abort;
   int maxhi;
@@ -125,22 +125,6 @@ struct TcShared {
   signed char xcol[kSelThreads];  // spare segment index, -1: none
   int pool;                 // spare segments handed out
 };
-
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag,
-                                              uint32_t* status) {
-  if (sm100::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = sm100::globaltimer_ns();
-  while (true) {
-    if (sm100::mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      raise_flag(status, kErrTimeout);
-      return false;
-    }
-  }
-}
 
 // Append (score, code) at the segment cursor when score >= L; predicated
 // stores, so a warp never branches on the comparison.
@@ -404,6 +388,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       sm100::mbar_init(&sh.kempty[s], 1);
     }
     sm100::mbar_init(&sh.qfull, 1);
+    sm100::mbar_init(&sh.never, 1);
     for (int t = 0; t < kTmemBufs; ++t) {
       sm100::mbar_init(&sh.tfull[t], 1);
       sm100::mbar_init(&sh.tempty[t], kSelWarps);
@@ -442,7 +427,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       for (int t = 0; t < TT; ++t) {
         const int tile = t < T ? t : t - T;
         if (t >= NS &&
-            !wait_or_abort(&sh.kempty[s], ph ^ 1, abort_flag, a.status))
+            !sm100::wait_or_abort(&sh.kempty[s], ph ^ 1, abort_flag, a.status,
+                                   a.wait_ns))
           break;
         sm100::mbar_arrive_expect_tx(&sh.kfull[s], Lay::kKBytes);
         unsigned char* dst = sK + (size_t)s * Lay::kKBytes;
@@ -456,9 +442,11 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         }
       }
       // Let every copy this thread started land before the CTA can exit.
-      sm100::mbar_wait(&sh.qfull, 0, kWaitLimitNs);
+      bool drained = sm100::mbar_wait(&sh.qfull, 0, kDrainWaitNs);
       for (int t = issued - NS < 0 ? 0 : issued - NS; t < issued; ++t)
-        sm100::mbar_wait(&sh.kfull[t % NS], (t / NS) & 1, kWaitLimitNs);
+        drained &= sm100::mbar_wait(&sh.kfull[t % NS], (t / NS) & 1,
+                                    kDrainWaitNs);
+      if (!drained) raise_flag(a.status, kErrTimeout);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -467,15 +455,23 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       const uint32_t aq = sm100::smem_u32(sQ);
       const uint32_t ak = sm100::smem_u32(sK);
       int done = 0;
-      if (wait_or_abort(&sh.qfull, 0, abort_flag, a.status)) {
+      if (a.stall_ns) {
+        // Failure-path test hook: wait on a barrier that nothing signals, so
+        // the wait runs out, raises the time-out flag and aborts every wait
+        // of the CTA; the kernel then leaves through its normal path.
+        sm100::wait_or_abort(&sh.never, 0, abort_flag, a.status, a.stall_ns);
+      }
+      if (sm100::wait_or_abort(&sh.qfull, 0, abort_flag, a.status, a.wait_ns)) {
         int s = 0;
         uint32_t ph = 0;
         for (int t = 0; t < TT; ++t) {
           const int buf = t & (kTmemBufs - 1);
-          if (!wait_or_abort(&sh.kfull[s], ph, abort_flag, a.status)) break;
+          if (!sm100::wait_or_abort(&sh.kfull[s], ph, abort_flag, a.status,
+                                    a.wait_ns))
+            break;
           if (t >= kTmemBufs &&
-              !wait_or_abort(&sh.tempty[buf], ((t / kTmemBufs) & 1) ^ 1,
-                             abort_flag, a.status))
+              !sm100::wait_or_abort(&sh.tempty[buf], ((t / kTmemBufs) & 1) ^ 1,
+                                    abort_flag, a.status, a.wait_ns))
             break;
           sm100::tc_fence_after();
           const uint32_t d_tmem = tmem + buf * BN;
@@ -496,9 +492,10 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         }
       }
       // The last commit covers every MMA issued: wait for it before exit.
-      if (done > 0)
-        sm100::mbar_wait(&sh.tfull[(done - 1) & (kTmemBufs - 1)],
-                         ((done - 1) / kTmemBufs) & 1, kWaitLimitNs);
+      if (done > 0 &&
+          !sm100::mbar_wait(&sh.tfull[(done - 1) & (kTmemBufs - 1)],
+                            ((done - 1) / kTmemBufs) & 1, kDrainWaitNs))
+        raise_flag(a.status, kErrTimeout);
     }
   } else {
     // ---------------- selector warps: thread = (query row, chunk group)
@@ -515,8 +512,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     auto fetch = [&](int t, uint32_t (&raw)[32]) -> bool {
       const int buf = t & (kTmemBufs - 1);
       if (!__all_sync(0xFFFFFFFFu,
-                      wait_or_abort(&sh.tfull[buf], (t / kTmemBufs) & 1,
-                                    abort_flag, a.status)))
+                      sm100::wait_or_abort(&sh.tfull[buf], (t / kTmemBufs) & 1,
+                                           abort_flag, a.status, a.wait_ns)))
         return false;
       sm100::tc_fence_after();
       sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
@@ -1513,8 +1510,7 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   if (Lay::bytes(P) > budget || P < 40) return cudaErrorNotSupported;
   const size_t smem = Lay::bytes(P);
   auto kern = prefill_score_topk_tc<D>;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_tc");
@@ -1525,7 +1521,7 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   // rows whose segments overflowed (rare on typical inputs): exact fallback
   const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
   prof_before(s, "prefill_overflow_rows");
-  prefill_overflow_rows<__nv_bfloat16, D><<<148, kFbThreads, fb_smem, s>>>(a);
+  prefill_overflow_rows<__nv_bfloat16, D><<<sm_count(), kFbThreads, fb_smem, s>>>(a);
   prof_after(s);
   return cudaGetLastError();
 }
@@ -1535,8 +1531,7 @@ cudaError_t launch_select_f32(const PrefillArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)32 * D * 4 + (size_t)a.k * kTileRows * 8 +
                       (size_t)32 * kTileRows * 8;
   auto kern = prefill_score_topk_f32<D>;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_f32");
@@ -1573,8 +1568,7 @@ cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
   auto k2 = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, 2>
                      : prefill_gather_mma<D, float, 2>;
   auto kern = a.k <= 32 ? k1 : k2;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   prof_before(s, "prefill_gather");
   kern<<<grid, kMmaWarps * 32, smem, s>>>(a);

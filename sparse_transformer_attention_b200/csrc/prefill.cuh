@@ -25,6 +25,8 @@ struct PrefillArgs {
   uint64_t* topk;    // [B*Hq*n, k] selected keys per row (workspace)
   uint32_t* ovf_count;  // rows listed for the exact fallback (status area)
   uint32_t* ovf_rows;   // [B*Hq*n] their row indices (workspace)
+  uint64_t wait_ns;     // limit of each pipeline wait (kPipelineWaitNs)
+  uint64_t stall_ns;    // failure-path test hook (0: off)
 };
 
 // Bytes of the per-row Top-k key area at the start of the workspace body.

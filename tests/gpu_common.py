@@ -60,12 +60,35 @@ def run_prefill(w, x, W_i=None, o_dtype=torch.float32):
                                              o_dtype=o_dtype)
     status = ca.condensate_attn_status(ws)
     assert status == ca.CA_OK, ca.status_string(status)
-    return O, idx, cnt, C_max
+    return O, idx, cnt, C_max, ws
 
 
-def check_prefill(w, x, W_i=None, sel=None, o_dtype=torch.float32, tol=None):
-    """Compare all rows (sel=None) or the sampled (b, h, i) rows `sel`."""
-    O, idx, cnt, C_max = run_prefill(w, x, W_i, o_dtype)
+def fallback_rows(w, ws):
+    """(b, h, i) of the rows the prefill selector listed for its exact
+    fallback pass (read from the workspace: the count sits in the status
+    area at byte 16, the row list after the per-row Top-k keys)."""
+    R = w.B * w.Hq * w.n
+    cnt = int(ws[16:20].cpu().numpy().view(np.uint32)[0])
+    topk_bytes = (R * max(w.k, 1) * 8 + 255) // 256 * 256
+    off = 256 + topk_bytes
+    rows = ws[off:off + 4 * cnt].cpu().numpy().view(np.uint32).astype(np.int64)
+    bh, i = np.divmod(rows, w.n)
+    b, h = np.divmod(bh, w.Hq)
+    return np.stack([b, h, i], 1).reshape(-1, 3)
+
+
+def check_prefill(w, x, W_i=None, sel=None, o_dtype=torch.float32, tol=None,
+                  with_fallback_rows=False):
+    """Compare all rows (sel=None) or the sampled (b, h, i) rows `sel`
+    (plus, with_fallback_rows, every row that took the exact fallback)."""
+    O, idx, cnt, C_max, ws = run_prefill(w, x, W_i, o_dtype)
+    nfb = 0
+    if with_fallback_rows:
+        fb = fallback_rows(w, ws)
+        nfb = len(fb)
+        if sel is not None:
+            sel = np.unique(np.concatenate([np.asarray(sel, np.int64), fb]),
+                            axis=0)
     if sel is None:
         b, h, i = np.meshgrid(np.arange(w.B), np.arange(w.Hq), np.arange(w.n),
                               indexing="ij")
@@ -79,10 +102,13 @@ def check_prefill(w, x, W_i=None, sel=None, o_dtype=torch.float32, tol=None):
                          C_max=C_max, with_full=False)
     G = w.Hq // w.Hkv
     win = [int(W_i[b, i]) if W_i is not None else w.W for (b, h, i) in sel]
-    return check_rows(
+    out = check_rows(
         ref, g_idx, g_cnt, g_o,
         q_rows=[x["Q"][b, h, i] for (b, h, i) in sel],
         kv_rows=lambda r: x["K"][sel[r][0], sel[r][1] // G],
         v_rows=lambda r: x["V"][sel[r][0], sel[r][1] // G],
         pos=sel[:, 2], win=win,
         tol=tol if tol is not None else TOL[w.dtype])
+    if with_fallback_rows:
+        out["fallback_rows"] = nfb
+    return out

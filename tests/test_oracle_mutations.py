@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_rounding_bound as rb
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "condensate_oracle.c")
 
@@ -36,6 +37,12 @@ MUTATIONS = {
     "normalisation_dropped": ("for (int l = 0; l < d; ++l) o[l] /= den;", ""),
     "all_candidates_one_short": ("int64_t m = k < ncand ? k : ncand;",
                                  "int64_t m = k < ncand ? k : ncand - 1;"),
+    "bound_unit_roundoff_too_small": ("double u = ldexp(1.0, -23);",
+                                      "double u = ldexp(1.0, -30);"),
+    "bound_unselected_term_dropped": ("diag[DG_BOUND] = gam * (amax_sel + amax_unsel);",
+                                      "diag[DG_BOUND] = gam * amax_sel;"),
+    "bound_ten_times_too_large": ("diag[DG_BOUND] = gam * (amax_sel + amax_unsel);",
+                                  "diag[DG_BOUND] = 10.0 * gam * (amax_sel + amax_unsel);"),
     "score_term_dropped": ("for (int l = 0; l < d; ++l) acc += (double)q[l] * (double)kj[l];",
                            "for (int l = 1; l < d; ++l) acc += (double)q[l] * (double)kj[l];"),
 }
@@ -50,6 +57,9 @@ PIN_TESTS = [
     pins.test_uniform_scores_closed_forms,
     pins.test_planted_needles_are_selected,
     pins.test_lemma_excluded_scores_below_threshold,
+    lambda: [rb.test_oracle_bound_covers_every_order(d, adv)
+             for d in (64, 128) for adv in (False, True)],
+    rb.test_oracle_bound_on_workload_rows,
 ]
 
 

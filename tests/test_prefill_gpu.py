@@ -66,18 +66,21 @@ def test_prefill_bf16_output():
                         tol=1e-2 + 2.0 ** -6))
 
 
-def test_prefill_gpt2s_8k_sampled():
-    """The GPT-2-small 8K prefill workload at full size, sampled rows."""
+def test_prefill_gpt2s_8k_all_rows():
+    """The GPT-2-small 8K prefill workload at full size, every one of its
+    393,216 rows (and any row that took the exact fallback among them)."""
     w = workloads.get("prefill_gpt2s_8k")
     x = workloads.generate(w)
-    print(check_prefill(w, x, sel=_sample_rows(w, 1500, 0)))
+    print(check_prefill(w, x, with_fallback_rows=True))
 
 
 def test_prefill_adaptive_32k_sampled():
-    """The adaptive-window 32K prefill workload at full size, sampled rows."""
+    """The adaptive-window 32K prefill workload at full size: 20,000 sampled
+    rows plus every row the selector sent to the exact fallback."""
     w = workloads.get("prefill_adaptive_32k")
     x = workloads.generate(w)
-    print(check_prefill(w, x, W_i=x["W_i"], sel=_sample_rows(w, 600, 1)))
+    print(check_prefill(w, x, W_i=x["W_i"], sel=_sample_rows(w, 20000, 1),
+                        with_fallback_rows=True))
 
 
 @pytest.mark.parametrize("d", [64, 128])

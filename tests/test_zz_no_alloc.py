@@ -28,13 +28,16 @@ def _p(t):
     return None if t is None else P(t.data_ptr())
 
 
-def _noalloc(lib, q, K, V, w, O, idx, cnt, C_max):
+def _stream():
+    return P(torch.cuda.current_stream().cuda_stream)
+
+
+def _noalloc(lib, q, K, V, w, O, idx, cnt, C_max, W_i=None):
     dt = binding.CA_BF16 if q.dtype == torch.bfloat16 else binding.CA_F32
     odt = binding.CA_BF16 if O.dtype == torch.bfloat16 else binding.CA_F32
     return lib.condensate_attn_decode_noalloc(
-        _p(q), _p(K), _p(V), dt, w.B, w.n, w.Hq, w.Hkv, w.d, w.W, w.k, None,
-        _p(O), odt, _p(idx), _p(cnt), C_max,
-        P(torch.cuda.current_stream().cuda_stream))
+        _p(q), _p(K), _p(V), dt, w.B, w.n, w.Hq, w.Hkv, w.d, w.W, w.k,
+        _p(W_i), _p(O), odt, _p(idx), _p(cnt), C_max, _stream())
 
 
 @pytest.mark.parametrize("dtype,tol", [("bf16", 1e-2), ("f32", 1e-5)])
@@ -59,6 +62,30 @@ def test_noalloc_matches_workspace_entry_point(dtype, tol):
         assert torch.equal(idx, idx_ref), call
         err = (O - O_ref).abs().max().item()
         assert err <= tol, (call, err)
+        # the built-in buffer's status word: nothing raised
+        assert lib.condensate_attn_decode_noalloc_status(_stream()) == \
+            binding.CA_OK, call
+
+
+def test_noalloc_status_reports_device_flags():
+    """A per-batch window below 1 is only seen on the device: the flag lands
+    in the built-in buffer and the status reader reports (and clears) it."""
+    lib = binding.load()
+    w = workloads.get("decode_131k").scaled(n=6000, B=2, Hq=8, Hkv=2,
+                                            needles=4)
+    x = workloads.generate(w)
+    q, K, V = (torch.from_numpy(x[n]).cuda().to(torch.bfloat16)
+               for n in ("Q", "K", "V"))
+    C_max = min(w.n, 1 + w.W + w.k)
+    O = torch.empty((w.B, w.Hq, w.d), device="cuda")
+    idx = torch.empty((w.B, w.Hq, C_max), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.B, w.Hq), dtype=torch.int32, device="cuda")
+    W_i = torch.tensor([w.W, 0], dtype=torch.int32, device="cuda")
+    assert _noalloc(lib, q, K, V, w, O, idx, cnt, C_max, W_i) == binding.CA_OK
+    assert lib.condensate_attn_decode_noalloc_status(_stream()) == \
+        binding.CA_ERR_DEVICE_ARG
+    assert lib.condensate_attn_decode_noalloc_status(_stream()) == \
+        binding.CA_OK
 
 
 def test_noalloc_rejects_problems_beyond_its_buffer():
