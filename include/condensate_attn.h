@@ -98,6 +98,37 @@ CA_API size_t condensate_attn_workspace_size(int is_decode, ca_dtype dtype, int 
                                       int W_max, int k);
 
 /*
+ * Optional inputs and outputs of the _ex entry points (all device pointers,
+ * each may be NULL; the struct itself may be NULL).
+ *
+ *   W_h   [Hq] int32: window of each q-head ("Condensate Theorem" page 1
+ *         §6 layer-wise window schedule and §10.2 per-head parameters: a
+ *         schedule over layers is one call per layer with its own W or W_h).
+ *         The window of row (b, h, i) is W_i[b, i] when W_i is given, else
+ *         W_h[h] when given, else W.  Values below 1 raise
+ *         CA_ERR_DEVICE_ARG and are read as 1.
+ *   k_h   [Hq] int32: Top-k size of each q-head, each in [0, k] (k, the
+ *         scalar argument, is the largest and sizes the workspace; k_h = 0
+ *         is the static anchor + window variant).  Values outside [0, k]
+ *         raise CA_ERR_DEVICE_ARG and are clamped.
+ *   mass  [rows, 4] fp32: per query row, over the full causal softmax
+ *         A_ij = softmax_j<=i(t_ij / sqrt(d)) (§2.2.1, §2.2.2, §3.2.2):
+ *           [0] anchor mass   A_i0
+ *           [1] window mass   sum over j in [max(0, i-W_i+1), i] of A_ij
+ *           [2] Top-k mass    sum over the selected Top-k of A_ij
+ *           [3] excluded mass epsilon_i = sum over causal j not in C_i
+ *   lse   [rows] fp32: log sum_j<=i exp(t_ij / sqrt(d)) (natural log).
+ * rows = B*Hq*nq for prefill, B*Hq for decode.  Asking for mass or lse adds
+ * one exponential per causal score to the score pass.
+ */
+typedef struct {
+  const int32_t* W_h;
+  const int32_t* k_h;
+  float* mass;
+  float* lse;
+} ca_extras;
+
+/*
  * Causal prefill over n positions (§2.1 Definition 1 applied to every row,
  * §5.2.2 select-then-attend).  Two launches: a fused score + Top-k pass
  * (tcgen05 tensor cores for bf16, FFMA for fp32) and a gather + fp32 online
@@ -113,6 +144,31 @@ CA_API ca_status condensate_attn_prefill(const void* Q, const void* K, const voi
                                   void* stream);
 
 /*
+ * Prefill of the last nq positions against an L-long cache (a chunk of a
+ * longer prefill, or several decode queries at once; §2.1 Definition 1 for
+ * rows L-nq .. L-1, §5.2.2).  Q [B, Hq, nq, d]; K, V [B, Hkv, L, d] with
+ * 1 <= nq <= L; query row r sits at position i = L - nq + r and attends to
+ * keys 0..i.  W_i is [B, nq]; outputs are [B, Hq, nq, ...].  nq = L is
+ * condensate_attn_prefill.  The workspace is
+ * condensate_attn_workspace_size_ex(0, dtype, B, nq, L, Hq, Hkv, d, W_max, k).
+ */
+CA_API ca_status condensate_attn_prefill_ex(
+    const void* Q, const void* K, const void* V, ca_dtype dtype, int B, int nq,
+    int L, int Hq, int Hkv, int d, int W, int k, const int32_t* W_i,
+    const ca_extras* extras, void* O, ca_dtype o_dtype, int32_t* idx,
+    int32_t* idx_count, int C_max, void* workspace, size_t workspace_bytes,
+    void* stream);
+
+/*
+ * Workspace bytes of condensate_attn_prefill_ex (is_decode = 0) or
+ * condensate_attn_decode_ex (is_decode = 1, nq = 1) with these sizes.
+ */
+CA_API size_t condensate_attn_workspace_size_ex(int is_decode, ca_dtype dtype,
+                                                int B, int nq, int L, int Hq,
+                                                int Hkv, int d, int W_max,
+                                                int k);
+
+/*
  * Decode of one query per (batch, q-head) at position L-1 against an L-long
  * cache (§2.1 Definition 1 for the last row).  Two launches: a K-streaming
  * score pass with a per-chunk Top-k, and a merge + gather + softmax pass.
@@ -125,6 +181,25 @@ CA_API ca_status condensate_attn_decode(const void* q, const void* K, const void
                                  int32_t* idx_count, int C_max,
                                  void* workspace, size_t workspace_bytes,
                                  void* stream);
+
+/*
+ * Number of key chunks the decode score pass splits an L-long cache into on
+ * the current device (about two CTAs per SM).  The decode workspace holds,
+ * after its 256-byte status area, the best k selection keys of every chunk
+ * and q-head, [B, Hq, chunks, k] 64-bit keys (fp32 score bits in an
+ * order-preserving form in the high word, 0xFFFFFFFF - position in the low
+ * word, 0 for an empty slot), in a 256-byte-rounded area.  For tests and
+ * debugging; 0 for invalid sizes.
+ */
+CA_API int condensate_attn_decode_chunks(int B, int L, int Hkv, int k);
+
+/* condensate_attn_decode with the optional inputs and outputs above. */
+CA_API ca_status condensate_attn_decode_ex(
+    const void* q, const void* K, const void* V, ca_dtype dtype, int B, int L,
+    int Hq, int Hkv, int d, int W, int k, const int32_t* W_i,
+    const ca_extras* extras, void* O, ca_dtype o_dtype, int32_t* idx,
+    int32_t* idx_count, int C_max, void* workspace, size_t workspace_bytes,
+    void* stream);
 
 /*
  * Decode without a workspace argument, for callers that cannot allocate

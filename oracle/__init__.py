@@ -26,7 +26,7 @@ _lib = None
 DIAG_NAMES = [
     "m", "size", "anchor_mass", "window_mass", "topk_mass", "excluded_mass",
     "cos", "err_l2", "vmax_l2", "tau_min", "best_unsel", "gap", "bound",
-    "win_lo",
+    "win_lo", "lse",
 ]
 
 

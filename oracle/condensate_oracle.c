@@ -59,6 +59,7 @@ enum {
   DG_GAP,              /* TAU_MIN - BEST_UNSEL (+inf if either is absent)  */
   DG_BOUND,            /* fp32 rounding bound beta_i on a score pair       */
   DG_WIN_LO,           /* first window position max(0, i-W_i+1)           */
+  DG_LSE,              /* log sum_{j<=i} exp(s_j): the softmax normaliser  */
   DG_COUNT
 };
 
@@ -240,6 +241,7 @@ int64_t oracle_row(const float* q, const float* K, const float* V, int d,
       A[j] = exp(t[j] * scale - mx);
       den += A[j];
     }
+    if (diag) diag[DG_LSE] = mx + log(den);
     for (int l = 0; l < d; ++l) o_full[l] = 0.0;
     double vmax = 0.0;
     for (int64_t j = 0; j < nkeys; ++j) {

@@ -29,9 +29,17 @@ CA_ERR_INTERNAL = 8
 CA_F32 = 0
 CA_BF16 = 1
 
+class CaExtras(ctypes.Structure):
+    """ca_extras of the header: optional per-head windows and Top-k sizes,
+    mass and log-sum-exp outputs (device pointers, NULL = unused)."""
+    _fields_ = [("W_h", ctypes.c_void_p), ("k_h", ctypes.c_void_p),
+                ("mass", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+
+
 # (name, restype, argtypes) of every entry point the header declares.
 _P = ctypes.c_void_p
 _I = ctypes.c_int
+_X = ctypes.POINTER(CaExtras)
 SIGNATURES = {
     "condensate_attn_workspace_size":
         (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
@@ -41,6 +49,15 @@ SIGNATURES = {
     "condensate_attn_decode":
         (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
               _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_workspace_size_ex":
+        (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "condensate_attn_prefill_ex":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _X, _P, _I,
+              _P, _P, _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_decode_ex":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _X, _P, _I, _P,
+              _P, _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_decode_chunks": (_I, [_I, _I, _I, _I]),
     "condensate_attn_decode_noalloc":
         (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
               _I, _P]),
@@ -124,6 +141,39 @@ def _require(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def condensate_attn_workspace_size_ex(is_decode: bool, dtype: torch.dtype,
+                                      B: int, nq: int, L: int, Hq: int,
+                                      Hkv: int, d: int, W_max: int,
+                                      k: int) -> int:
+    return int(load().condensate_attn_workspace_size_ex(
+        int(bool(is_decode)), _dt(dtype), B, nq, L, Hq, Hkv, d, W_max, k))
+
+
+def _extras(W_h, k_h, mass, lse):
+    if W_h is None and k_h is None and mass is None and lse is None:
+        return None
+    for t, nm in ((W_h, "W_h"), (k_h, "k_h"), (mass, "mass"), (lse, "lse")):
+        if t is not None:
+            _require(t, nm)
+    for t, nm in ((W_h, "W_h"), (k_h, "k_h")):
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError(f"{nm} must be int32")
+    for t, nm in ((mass, "mass"), (lse, "lse")):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{nm} must be float32")
+    x = CaExtras(_ptr(W_h), _ptr(k_h), _ptr(mass), _ptr(lse))
+    return ctypes.byref(x), x
+
+
+def _w_max(W, W_i, W_h):
+    m = [int(W)]
+    if W_i is not None:
+        m = [int(W_i.max().item())]
+    elif W_h is not None:
+        m = [int(W_h.max().item())]
+    return max(1, m[0])
+
+
 def condensate_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                             W: int, k: int, W_i: Optional[torch.Tensor] = None,
                             O: Optional[torch.Tensor] = None,
@@ -132,35 +182,44 @@ def condensate_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                             idx_count: Optional[torch.Tensor] = None,
                             C_max: Optional[int] = None,
                             workspace: Optional[torch.Tensor] = None,
-                            stream=None) -> Tuple[torch.Tensor, torch.Tensor,
-                                                  torch.Tensor]:
-    """Causal prefill.  Q [B,Hq,n,d], K/V [B,Hkv,n,d] (fp32 or bf16, CUDA).
+                            stream=None, W_h: Optional[torch.Tensor] = None,
+                            k_h: Optional[torch.Tensor] = None,
+                            mass: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None
+                            ) -> Tuple[torch.Tensor, torch.Tensor,
+                                       torch.Tensor]:
+    """Causal prefill.  Q [B,Hq,nq,d], K/V [B,Hkv,L,d] (fp32 or bf16, CUDA)
+    with nq <= L: query row r sits at position L - nq + r (nq = L is a full
+    prefill).  W_i [B,nq], W_h [Hq], k_h [Hq] (int32) are optional; mass
+    [B,Hq,nq,4] and lse [B,Hq,nq] (float32) are optional outputs.
 
-    Returns (O [B,Hq,n,d], idx [B,Hq,n,C_max] int32, idx_count [B,Hq,n]).
+    Returns (O [B,Hq,nq,d], idx [B,Hq,nq,C_max] int32, idx_count [B,Hq,nq]).
     """
-    B, Hq, n, d = Q.shape
-    Hkv = K.shape[1]
+    B, Hq, nq, d = Q.shape
+    Hkv, L = K.shape[1], K.shape[2]
     for t, nm in ((Q, "Q"), (K, "K"), (V, "V")):
         _require(t, nm)
-    W_max = int(W_i.max().item()) if (W_i is not None and C_max is None) else W
+    W_max = _w_max(W, W_i, W_h)
     if C_max is None:
-        C_max = 1 + W_max + k
+        C_max = min(L, 1 + W_max + k)
     dev = Q.device
     if O is None:
-        O = torch.empty((B, Hq, n, d), dtype=o_dtype, device=dev)
+        O = torch.empty((B, Hq, nq, d), dtype=o_dtype, device=dev)
     if idx is None:
-        idx = torch.empty((B, Hq, n, C_max), dtype=torch.int32, device=dev)
+        idx = torch.empty((B, Hq, nq, C_max), dtype=torch.int32, device=dev)
     if idx_count is None:
-        idx_count = torch.empty((B, Hq, n), dtype=torch.int32, device=dev)
+        idx_count = torch.empty((B, Hq, nq), dtype=torch.int32, device=dev)
     if workspace is None:
-        ws = condensate_attn_workspace_size(False, Q.dtype, B, n, Hq, Hkv, d,
-                                            max(1, W_max), k)
+        ws = condensate_attn_workspace_size_ex(False, Q.dtype, B, nq, L, Hq,
+                                               Hkv, d, W_max, k)
         workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
-    code = load().condensate_attn_prefill(
-        _ptr(Q), _ptr(K), _ptr(V), _dt(Q.dtype), B, n, Hq, Hkv, d, int(W),
-        int(k), _ptr(W_i), _ptr(O), _dt(O.dtype), _ptr(idx), _ptr(idx_count),
-        int(C_max), _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(code, "condensate_attn_prefill")
+    ex = _extras(W_h, k_h, mass, lse)
+    code = load().condensate_attn_prefill_ex(
+        _ptr(Q), _ptr(K), _ptr(V), _dt(Q.dtype), B, nq, L, Hq, Hkv, d, int(W),
+        int(k), _ptr(W_i), ex[0] if ex else None, _ptr(O), _dt(O.dtype),
+        _ptr(idx), _ptr(idx_count), int(C_max), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_prefill_ex")
     return O, idx, idx_count
 
 
@@ -172,9 +231,15 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                            idx_count: Optional[torch.Tensor] = None,
                            C_max: Optional[int] = None,
                            workspace: Optional[torch.Tensor] = None,
-                           stream=None) -> Tuple[torch.Tensor, torch.Tensor,
-                                                 torch.Tensor]:
-    """Decode at position L-1.  q [B,Hq,d], K/V [B,Hkv,L,d] (CUDA).
+                           stream=None, W_h: Optional[torch.Tensor] = None,
+                           k_h: Optional[torch.Tensor] = None,
+                           mass: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor,
+                                      torch.Tensor]:
+    """Decode at position L-1.  q [B,Hq,d], K/V [B,Hkv,L,d] (CUDA).  W_i [B],
+    W_h [Hq], k_h [Hq] (int32) optional; mass [B,Hq,4], lse [B,Hq] optional
+    float32 outputs.
 
     Returns (O [B,Hq,d], idx [B,Hq,C_max] int32, idx_count [B,Hq]).
     """
@@ -182,7 +247,7 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     Hkv, L = K.shape[1], K.shape[2]
     for t, nm in ((q, "q"), (K, "K"), (V, "V")):
         _require(t, nm)
-    W_max = int(W_i.max().item()) if (W_i is not None and C_max is None) else W
+    W_max = _w_max(W, W_i, W_h)
     if C_max is None:
         C_max = min(L, 1 + W_max + k)
     dev = q.device
@@ -194,14 +259,21 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         idx_count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
     if workspace is None:
         ws = condensate_attn_workspace_size(True, q.dtype, B, L, Hq, Hkv, d,
-                                            max(1, W_max), k)
+                                            W_max, k)
         workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
-    code = load().condensate_attn_decode(
+    ex = _extras(W_h, k_h, mass, lse)
+    code = load().condensate_attn_decode_ex(
         _ptr(q), _ptr(K), _ptr(V), _dt(q.dtype), B, L, Hq, Hkv, d, int(W),
-        int(k), _ptr(W_i), _ptr(O), _dt(O.dtype), _ptr(idx), _ptr(idx_count),
-        int(C_max), _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(code, "condensate_attn_decode")
+        int(k), _ptr(W_i), ex[0] if ex else None, _ptr(O), _dt(O.dtype),
+        _ptr(idx), _ptr(idx_count), int(C_max), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_decode_ex")
     return O, idx, idx_count
+
+
+def condensate_attn_decode_chunks(B: int, L: int, Hkv: int, k: int) -> int:
+    """Key chunks of the decode score pass on the current device."""
+    return int(load().condensate_attn_decode_chunks(B, L, Hkv, k))
 
 
 def condensate_attn_status(workspace: torch.Tensor, stream=None) -> int:

@@ -30,17 +30,67 @@ bool group_ok(int Hq, int Hkv) {
   return G == 1 || G == 2 || G == 4 || G == 8;
 }
 
+// Decode workspace: status area | chunk lists [B, Hq, chunks, k] (64-bit
+// keys) | per-chunk candidate (max, sum) [B, Hq, chunks] (float2).
+size_t decode_lists_bytes(int B, int Hq, int nch, int k) {
+  return round_up((size_t)B * Hq * nch * (k > 0 ? k : 1) * 8, 256);
+}
 size_t decode_ws(int B, int L, int Hq, int Hkv, int k) {
-  int nch = ca::decode_chunks(B, L, Hkv, k);
-  return ca::kStatusBytes +
-         round_up((size_t)B * Hq * nch * (k > 0 ? k : 1) * 8, 256);
+  const int nch = ca::decode_chunks(B, L, Hkv, k);
+  return ca::kStatusBytes + decode_lists_bytes(B, Hq, nch, k) +
+         round_up((size_t)B * Hq * nch * 8, 256);
+}
+
+size_t prefill_ws(int B, int nq, int Hq, int k) {
+  return ca::kStatusBytes + ca::prefill_workspace((int64_t)B * Hq * nq, k);
+}
+
+bool sizes_ok(ca_dtype dtype, int B, int nq, int L, int Hq, int Hkv, int d,
+              int W_max, int k) {
+  return B >= 1 && nq >= 1 && L >= nq && group_ok(Hq, Hkv) && W_max >= 1 &&
+         k >= 0 && (d == 64 || d == 128) &&
+         (dtype == CA_F32 || dtype == CA_BF16);
+}
+
+const ca_extras kNoExtras = {nullptr, nullptr, nullptr, nullptr};
+
+// Checks shared by every entry point, in the order the header lists them.
+ca_status check_common(const void* q, const void* K, const void* V,
+                       ca_dtype dtype, int B, int nq, int L, int Hq, int Hkv,
+                       int d, int W, int k, const int32_t* W_i,
+                       const ca_extras& x, void* O, ca_dtype o_dtype,
+                       int32_t* idx, int32_t* idx_count, int C_max, void* ws) {
+  if (!q || !K || !V || !O || !idx || !idx_count) return CA_ERR_INVALID_ARG;
+  if (B < 1 || nq < 1 || L < nq || k < 0 || C_max < 1)
+    return CA_ERR_INVALID_ARG;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return CA_ERR_INVALID_ARG;
+  const bool device_windows = W_i || x.W_h;
+  if (!device_windows && W < 1) return CA_ERR_INVALID_ARG;
+  if (!device_windows) {
+    // the largest set is the last row's: min(L, 1 + W + k)
+    long long need = 1LL + W + k;
+    if (need > L) need = L;
+    if (C_max < need) return CA_ERR_INVALID_ARG;
+  }
+  if (dtype != CA_F32 && dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
+  if (o_dtype != CA_F32 && o_dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return CA_ERR_UNSUPPORTED;
+  if (!group_ok(Hq, Hkv)) return CA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      !aligned16(idx) || !aligned16(idx_count) || !aligned16(ws) ||
+      (W_i && ((uintptr_t)W_i & 3u)) || (x.W_h && ((uintptr_t)x.W_h & 3u)) ||
+      (x.k_h && ((uintptr_t)x.k_h & 3u)) ||
+      (x.mass && ((uintptr_t)x.mass & 15u)) ||
+      (x.lse && ((uintptr_t)x.lse & 3u)))
+    return CA_ERR_ALIGNMENT;
+  return CA_OK;
 }
 
 }  // namespace
 
 extern "C" {
 
-int condensate_attn_version(void) { return 100; }
+int condensate_attn_version(void) { return 200; }
 
 const char* condensate_attn_status_string(ca_status s) {
   switch (s) {
@@ -57,52 +107,40 @@ const char* condensate_attn_status_string(ca_status s) {
   return "unknown status";
 }
 
+size_t condensate_attn_workspace_size_ex(int is_decode, ca_dtype dtype, int B,
+                                         int nq, int L, int Hq, int Hkv, int d,
+                                         int W_max, int k) {
+  if (is_decode) nq = 1;
+  if (!sizes_ok(dtype, B, nq, L, Hq, Hkv, d, W_max, k)) return 0;
+  if (is_decode) return decode_ws(B, L, Hq, Hkv, k);
+  return prefill_ws(B, nq, Hq, k);
+}
+
 size_t condensate_attn_workspace_size(int is_decode, ca_dtype dtype, int B,
                                       int n_or_L, int Hq, int Hkv, int d,
                                       int W_max, int k) {
-  if (B < 1 || n_or_L < 1 || !group_ok(Hq, Hkv) || W_max < 1 || k < 0 ||
-      (d != 64 && d != 128) || (dtype != CA_F32 && dtype != CA_BF16))
-    return 0;
-  if (is_decode) return decode_ws(B, n_or_L, Hq, Hkv, k);
-  return ca::kStatusBytes + ca::prefill_workspace(dtype == CA_BF16, B, n_or_L,
-                                                  Hq, Hkv, d, k);
+  return condensate_attn_workspace_size_ex(is_decode, dtype, B, n_or_L,
+                                           n_or_L, Hq, Hkv, d, W_max, k);
 }
 
-static ca_status check_common(const void* q, const void* K, const void* V,
-                              ca_dtype dtype, int B, int n, int Hq, int Hkv,
-                              int d, int W, int k, const int32_t* W_i, void* O,
-                              ca_dtype o_dtype, int32_t* idx,
-                              int32_t* idx_count, int C_max, void* ws) {
-  if (!q || !K || !V || !O || !idx || !idx_count) return CA_ERR_INVALID_ARG;
-  if (B < 1 || n < 1 || k < 0 || C_max < 1) return CA_ERR_INVALID_ARG;
-  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return CA_ERR_INVALID_ARG;
-  if (!W_i && W < 1) return CA_ERR_INVALID_ARG;
-  if (!W_i) {
-    long long need = 1LL + W + k;
-    if (need > n) need = n;
-    if (C_max < need) return CA_ERR_INVALID_ARG;
-  }
-  if (dtype != CA_F32 && dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
-  if (o_dtype != CA_F32 && o_dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return CA_ERR_UNSUPPORTED;
-  if (!group_ok(Hq, Hkv)) return CA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
-      !aligned16(idx) || !aligned16(idx_count) || !aligned16(ws) ||
-      (W_i && ((uintptr_t)W_i & 3u)))
-    return CA_ERR_ALIGNMENT;
-  return CA_OK;
+int condensate_attn_decode_chunks(int B, int L, int Hkv, int k) {
+  if (B < 1 || L < 1 || Hkv < 1 || k < 0) return 0;
+  return ca::decode_chunks(B, L, Hkv, k);
 }
 
-ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
-                                 ca_dtype dtype, int B, int L, int Hq, int Hkv,
-                                 int d, int W, int k, const int32_t* W_i,
-                                 void* O, ca_dtype o_dtype, int32_t* idx,
-                                 int32_t* idx_count, int C_max,
-                                 void* workspace, size_t workspace_bytes,
-                                 void* stream) {
+ca_status condensate_attn_decode_ex(const void* q, const void* K,
+                                    const void* V, ca_dtype dtype, int B,
+                                    int L, int Hq, int Hkv, int d, int W,
+                                    int k, const int32_t* W_i,
+                                    const ca_extras* extras, void* O,
+                                    ca_dtype o_dtype, int32_t* idx,
+                                    int32_t* idx_count, int C_max,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream) {
   if (!workspace) return CA_ERR_WORKSPACE;
-  ca_status st = check_common(q, K, V, dtype, B, L, Hq, Hkv, d, W, k, W_i, O,
-                              o_dtype, idx, idx_count, C_max, workspace);
+  const ca_extras& x = extras ? *extras : kNoExtras;
+  ca_status st = check_common(q, K, V, dtype, B, 1, L, Hq, Hkv, d, W, k, W_i,
+                              x, O, o_dtype, idx, idx_count, C_max, workspace);
   if (st != CA_OK) return st;
   if (k > ca::kDecodeMaxK) return CA_ERR_UNSUPPORTED;
   if (workspace_bytes < decode_ws(B, L, Hq, Hkv, k)) return CA_ERR_WORKSPACE;
@@ -112,16 +150,70 @@ ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
   ca::DecodeArgs a;
   a.q = q; a.K = K; a.V = V;
   a.B = B; a.L = L; a.Hq = Hq; a.Hkv = Hkv; a.W = W; a.k = k;
-  a.W_i = W_i; a.O = O; a.o_bf16 = o_dtype == CA_BF16;
+  a.W_i = W_i; a.W_h = x.W_h; a.k_h = x.k_h; a.mass = x.mass; a.lse = x.lse;
+  a.O = O; a.o_bf16 = o_dtype == CA_BF16;
   a.idx = idx; a.idx_count = idx_count; a.C_max = C_max;
   a.nchunks = ca::decode_chunks(B, L, Hkv, k);
   a.chunk_len = ca::decode_chunk_len(L, a.nchunks);
   a.kpow2 = next_pow2(k > 1 ? k : 2);
   a.status = (uint32_t*)workspace;
   a.cand = (uint64_t*)((char*)workspace + ca::kStatusBytes);
+  a.cand_ml = (float2*)((char*)a.cand +
+                        decode_lists_bytes(B, Hq, a.nchunks, k));
   a.wait_ns = ca::kPipelineWaitNs;
   a.stall_ns = g_stall_ns.load();
   cudaError_t e = ca::decode_launch(a, dtype == CA_BF16, d, s);
+  return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+}
+
+ca_status condensate_attn_decode(const void* q, const void* K, const void* V,
+                                 ca_dtype dtype, int B, int L, int Hq, int Hkv,
+                                 int d, int W, int k, const int32_t* W_i,
+                                 void* O, ca_dtype o_dtype, int32_t* idx,
+                                 int32_t* idx_count, int C_max,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  return condensate_attn_decode_ex(q, K, V, dtype, B, L, Hq, Hkv, d, W, k, W_i,
+                                   nullptr, O, o_dtype, idx, idx_count, C_max,
+                                   workspace, workspace_bytes, stream);
+}
+
+ca_status condensate_attn_prefill_ex(const void* Q, const void* K,
+                                     const void* V, ca_dtype dtype, int B,
+                                     int nq, int L, int Hq, int Hkv, int d,
+                                     int W, int k, const int32_t* W_i,
+                                     const ca_extras* extras, void* O,
+                                     ca_dtype o_dtype, int32_t* idx,
+                                     int32_t* idx_count, int C_max,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!workspace) return CA_ERR_WORKSPACE;
+  const ca_extras& x = extras ? *extras : kNoExtras;
+  ca_status st = check_common(Q, K, V, dtype, B, nq, L, Hq, Hkv, d, W, k, W_i,
+                              x, O, o_dtype, idx, idx_count, C_max, workspace);
+  if (st != CA_OK) return st;
+  if (k > ca::kPrefillMaxK) return CA_ERR_UNSUPPORTED;
+  if (workspace_bytes < prefill_ws(B, nq, Hq, k)) return CA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, ca::kStatusBytes, s) != cudaSuccess)
+    return CA_ERR_CUDA;
+  const int64_t rows = (int64_t)B * Hq * nq;
+  ca::PrefillArgs a;
+  a.Q = Q; a.K = K; a.V = V;
+  a.B = B; a.nq = nq; a.L = L; a.p0 = L - nq;
+  a.Hq = Hq; a.Hkv = Hkv; a.W = W; a.k = k;
+  a.W_i = W_i; a.W_h = x.W_h; a.k_h = x.k_h; a.mass = x.mass; a.lse = x.lse;
+  a.O = O; a.o_bf16 = o_dtype == CA_BF16;
+  a.idx = idx; a.idx_count = idx_count; a.C_max = C_max;
+  a.status = (uint32_t*)workspace;
+  a.ovf_count = (uint32_t*)workspace + 4;  // inside the cleared status area
+  a.topk = (uint64_t*)((char*)workspace + ca::kStatusBytes);
+  a.ovf_rows = (uint32_t*)((char*)a.topk + ca::prefill_topk_bytes(rows, k));
+  a.cand_ml = (float2*)((char*)a.ovf_rows + round_up((size_t)rows * 4, 256));
+  a.wait_ns = ca::kPipelineWaitNs;
+  a.stall_ns = g_stall_ns.load();
+  cudaError_t e = ca::prefill_launch(a, dtype == CA_BF16, d, s);
+  if (e == cudaErrorNotSupported) return CA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
 }
 
@@ -133,31 +225,9 @@ ca_status condensate_attn_prefill(const void* Q, const void* K, const void* V,
                                   int32_t* idx_count, int C_max,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream) {
-  if (!workspace) return CA_ERR_WORKSPACE;
-  ca_status st = check_common(Q, K, V, dtype, B, n, Hq, Hkv, d, W, k, W_i, O,
-                              o_dtype, idx, idx_count, C_max, workspace);
-  if (st != CA_OK) return st;
-  if (k > ca::kPrefillMaxK) return CA_ERR_UNSUPPORTED;
-  size_t need = ca::kStatusBytes +
-                ca::prefill_workspace(dtype == CA_BF16, B, n, Hq, Hkv, d, k);
-  if (workspace_bytes < need) return CA_ERR_WORKSPACE;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemsetAsync(workspace, 0, ca::kStatusBytes, s) != cudaSuccess)
-    return CA_ERR_CUDA;
-  ca::PrefillArgs a;
-  a.Q = Q; a.K = K; a.V = V;
-  a.B = B; a.n = n; a.Hq = Hq; a.Hkv = Hkv; a.W = W; a.k = k;
-  a.W_i = W_i; a.O = O; a.o_bf16 = o_dtype == CA_BF16;
-  a.idx = idx; a.idx_count = idx_count; a.C_max = C_max;
-  a.status = (uint32_t*)workspace;
-  a.ovf_count = (uint32_t*)workspace + 4;  // inside the cleared status area
-  a.topk = (uint64_t*)((char*)workspace + ca::kStatusBytes);
-  a.ovf_rows = (uint32_t*)((char*)a.topk + ca::prefill_topk_bytes(B, n, Hq, k));
-  a.wait_ns = ca::kPipelineWaitNs;
-  a.stall_ns = g_stall_ns.load();
-  cudaError_t e = ca::prefill_launch(a, dtype == CA_BF16, d, s);
-  if (e == cudaErrorNotSupported) return CA_ERR_UNSUPPORTED;
-  return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+  return condensate_attn_prefill_ex(Q, K, V, dtype, B, n, n, Hq, Hkv, d, W, k,
+                                    W_i, nullptr, O, o_dtype, idx, idx_count,
+                                    C_max, workspace, workspace_bytes, stream);
 }
 
 ca_status condensate_attn_status(void* workspace, void* stream) {

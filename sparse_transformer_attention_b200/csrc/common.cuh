@@ -8,7 +8,7 @@
 namespace ca {
 
 // Bits of the device status word (first 4 bytes of the workspace).
-constexpr uint32_t kErrWindow = 1u;    // W_i outside [1, n or L]
+constexpr uint32_t kErrWindow = 1u;    // a window below 1 or k_h outside [0, k]
 constexpr uint32_t kErrTimeout = 2u;   // a bounded wait ran out
 constexpr uint32_t kErrCmax = 4u;      // |C_i| larger than C_max
 constexpr uint32_t kErrInternal = 8u;  // internal capacity check failed
@@ -121,18 +121,86 @@ template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat
   *p = __float2bfloat16_rn(v);
 }
 
-// Window of a query row: W_i[row] when given, else W.  A window below 1
-// raises kErrWindow and is read as 1; a window beyond `limit` (the sequence
-// or cache length) covers every causal position and is read as `limit`.
-__device__ __forceinline__ int row_window(const int32_t* W_i, int64_t row, int W,
+// Window of a query row: W_i[wi] when given, else W_h[h] when given, else
+// W.  A window below 1 raises kErrWindow (when `report`) and is read as 1;
+// a window beyond `limit` (the cache length) covers every causal position
+// and is read as `limit`.
+__device__ __forceinline__ int row_window(const int32_t* W_i, int64_t wi,
+                                          const int32_t* W_h, int h, int W,
                                           int limit, uint32_t* status,
                                           bool report) {
-  int w = W_i ? W_i[row] : W;
+  int w = W_i ? W_i[wi] : (W_h ? W_h[h] : W);
   if (w < 1) {
     if (report) raise_flag(status, kErrWindow);
     w = 1;
   }
   return w > limit ? limit : w;
+}
+
+// Top-k size of q-head h: k_h[h] when given (clamped to [0, k], a value
+// outside raising kErrWindow when `report`), else k.
+__device__ __forceinline__ int head_k(const int32_t* k_h, int h, int k,
+                                      uint32_t* status, bool report) {
+  if (!k_h) return k;
+  int kh = k_h[h];
+  if (kh < 0 || kh > k) {
+    if (report) raise_flag(status, kErrWindow);
+    kh = kh < 0 ? 0 : k;
+  }
+  return kh;
+}
+
+// Online log-sum-exp state in log2 units: the sum of 2^(x - m) over the
+// values x folded in, with m their maximum (m = -inf, l = 0 when empty).
+struct Lse2 {
+  float m = -INFINITY, l = 0.f;
+  __device__ __forceinline__ void add(float x) {
+    if (x > m) {
+      l = l * exp2f(m - x) + 1.f;
+      m = x;
+    } else {
+      l += exp2f(x - m);
+    }
+  }
+  __device__ __forceinline__ void merge(float m2, float l2) {
+    if (l2 == 0.f) return;
+    if (l == 0.f) {
+      m = m2;
+      l = l2;
+      return;
+    }
+    const float mn = fmaxf(m, m2);
+    l = l * exp2f(m - mn) + l2 * exp2f(m2 - mn);
+    m = mn;
+  }
+};
+
+// Mass report of one query row over the full causal softmax, from three
+// log2-domain (max, sum) states of scaled scores: C_i (m_c, l_c), the
+// window together with the anchor (m_wa, l_wa), and every candidate
+// [1, i-W_i] (m_cand, l_cand; the Top-k members are among them), plus the
+// anchor's own scaled score s0 (`anc`: the anchor lies outside the window).
+// Writes anchor, window, Top-k and excluded mass and the natural-log
+// log-sum-exp ("Condensate Theorem" page 1 §2.2.1, §2.2.2, §3.2.2).
+__device__ __forceinline__ void mass_report(float* mass, float* lse,
+                                            size_t row, float m_c, float l_c,
+                                            float m_wa, float l_wa,
+                                            float m_cand, float l_cand,
+                                            float s0, bool anc) {
+  const float F = l_cand > 0.f ? fmaxf(m_c, m_cand) : m_c;
+  const float lC = l_c * exp2f(m_c - F);
+  const float lwa = l_wa > 0.f ? l_wa * exp2f(m_wa - F) : 0.f;
+  const float lcand = l_cand > 0.f ? l_cand * exp2f(m_cand - F) : 0.f;
+  const float p0 = exp2f(s0 - F);
+  const float all = lwa + lcand;
+  const float ltop = fmaxf(lC - lwa, 0.f);
+  if (mass) {
+    mass[row * 4 + 0] = p0 / all;
+    mass[row * 4 + 1] = fmaxf(lwa - (anc ? p0 : 0.f), 0.f) / all;
+    mass[row * 4 + 2] = ltop / all;
+    mass[row * 4 + 3] = fmaxf(lcand - ltop, 0.f) / all;
+  }
+  if (lse) lse[row] = (F + log2f(all)) * 0.6931471805599453f;
 }
 
 }  // namespace ca

@@ -101,8 +101,12 @@ struct TopkShared {
   uint64_t never;  // failure-path test hook: a barrier nothing signals
   uint64_t thr[G];
   int cnt[G];
+  int kk[G];       // Top-k size of each q-head of the group
+  int hi[G];       // last candidate position of each q-head
   int abort;
   uint32_t hist[G][256];  // one radix histogram per list (per cutting warp)
+  float2 ml[8][G];        // per compute warp and head: (max, sum) of the
+                          // candidates' log2-scaled scores (mass reports)
 };
 
 // One warp cuts the list lst[0..n) of unique keys down to its best kk keys
@@ -179,20 +183,27 @@ __device__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint32_t* hist,
 }
 
 // At a check point (all inserts of the stretch done): warp h cuts list h
-// when it holds more than `limit` keys.  Barriers on both sides keep every
-// compute warp from inserting while a list is being cut.
+// down to its head's k keys when it holds more than the limit: that k after
+// the first stretch (so that a useful threshold exists early), else the
+// insert room the next stretch needs (`later`: long chunks also cut once a
+// list passes 4k keys, which raises the admission threshold early).
+// Barriers on both sides keep every compute warp from inserting while a list
+// is being cut.
 template <int G>
-__device__ __forceinline__ void check_lists(uint64_t* buf, int cap, int k,
-                                            int limit, TopkShared<G>* sh,
+__device__ __forceinline__ void check_lists(uint64_t* buf, int cap, bool first,
+                                            bool long_chunk, TopkShared<G>* sh,
                                             int warp, int lane) {
   ComputeBar::sync();
   if (warp < G) {
     const int n = sh->cnt[warp];
-    if (n > limit && n > k) {
-      const uint64_t T = warp_cut(buf + (size_t)warp * cap, n, k,
+    const int kk = sh->kk[warp];
+    const int limit = first ? kk
+                      : (long_chunk ? min(cap - kSub, 4 * kk) : cap - kSub);
+    if (kk > 0 && n > limit && n > kk) {
+      const uint64_t T = warp_cut(buf + (size_t)warp * cap, n, kk,
                                   sh->hist[warp], lane);
       if (lane == 0) {
-        sh->cnt[warp] = k;
+        sh->cnt[warp] = kk;
         sh->thr[warp] = T;
       }
     }
@@ -233,7 +244,7 @@ __device__ __forceinline__ void pairs16<float>(const uint4& v, float2* p) {
   p[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool MASS>
 __global__ void __launch_bounds__(kThreads, G >= 8 ? 1 : 2)
 decode_score_topk(DecodeArgs a) {
   using C = ScoreCfg<T, D, G>;
@@ -252,9 +263,22 @@ decode_score_topk(DecodeArgs a) {
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L;  // positions fit in 31 bits (int L in the ABI)
-  const int Wb = row_window(a.W_i, b, a.W, L, a.status,
-                            chunk == 0 && g == 0 && tid == 0);
-  const int hi = (L - 1) - Wb;  // last candidate position
+  // per q-head of the group: window (W_i per batch, else W_h per head, else
+  // W), last candidate position and Top-k size; the CTA streams up to the
+  // largest last candidate position of the group
+  int hi = -1;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const int hq = g * G + h;
+    const bool rep = chunk == 0 && tid == 0;
+    const int hh = (L - 1) - row_window(a.W_i, b, a.W_h, hq, a.W, L,
+                                        a.status, rep);
+    hi = max(hi, hh);
+    if (tid == 0) {
+      sh->hi[h] = hh;
+      sh->kk[h] = head_k(a.k_h, hq, a.k, a.status, rep);
+    }
+  }
   const int j0 = chunk * a.chunk_len;
   const int c0 = j0 < 1 ? 1 : j0;
   const int c1 = (j0 + a.chunk_len < hi + 1) ? j0 + a.chunk_len : hi + 1;
@@ -271,7 +295,8 @@ decode_score_topk(DecodeArgs a) {
     sm100::mbar_init(&sh->never, 1);
     for (int h = 0; h < G; ++h) {
       sh->cnt[h] = 0;
-      sh->thr[h] = 0ull;
+      // a head with k = 0 admits nothing
+      sh->thr[h] = sh->kk[h] > 0 ? 0ull : ~0ull;
     }
     sh->abort = 0;
     sm100::fence_barrier_init();
@@ -333,12 +358,14 @@ decode_score_topk(DecodeArgs a) {
   }
   const int myh = reduce_head<G>(l8);
   const bool owner = reduce_owner<G>(l8);
+  const int my_hi = sh->hi[myh];
   // Long chunks cut their lists again once they pass 4k keys, which raises
   // the admission threshold early (measured: 1M context 5% faster); short
   // chunks cut only when a list runs out of room (131K: the extra cuts cost
   // more than they save).
-  const int later_limit =
-      a.chunk_len >= 16 * kSub ? min(cap - kSub, 4 * k) : cap - kSub;
+  const bool long_chunk = a.chunk_len >= 16 * kSub;
+  const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e)/sqrt(d)
+  Lse2 ml;                   // candidates' scaled scores (mass reports)
   uint64_t thr = 0ull;       // admission threshold key (0: admit all)
   float thr_f = -INFINITY;   // its score, for a cheap float pre-filter
   const int first_keys = nrows < kSub ? nrows : kSub;
@@ -383,14 +410,19 @@ decode_score_topk(DecodeArgs a) {
 #pragma unroll
         for (int h = 0; h < G; ++h) part[h] = acc[h].x + acc[h].y;
         const float sc = group_reduce<G>(part, lane);
+        if constexpr (MASS) {
+          if (owner && j < c1 && j <= my_hi) ml.add(sc * sl2);
+        }
         if (t < C::SUB_ST) {
-          // first stretch: every key goes in, at its own slot
+          // first stretch: every key goes in, at its own slot (a position
+          // past this head's window start goes in as an empty key)
           if (owner && j < c1)
-            buf[(size_t)myh * cap + (j - c0)] = make_key(sc, (uint32_t)j);
+            buf[(size_t)myh * cap + (j - c0)] =
+                j <= my_hi ? make_key(sc, (uint32_t)j) : 0ull;
         } else {
           // rare once a threshold exists (a warp vote in front of this
           // branch measured slower)
-          const bool cand = owner && j < c1 && sc >= thr_f;
+          const bool cand = owner && j < c1 && j <= my_hi && sc >= thr_f;
           if (cand) {
             const uint64_t key = make_key(sc, (uint32_t)j);
             if (key > thr) {
@@ -411,15 +443,34 @@ decode_score_topk(DecodeArgs a) {
       if (t < C::SUB_ST) {
         // the first stretch filled slots 0..first_keys-1 of every list
         ComputeBar::sync();
-        if (tid < G) sh->cnt[tid] = first_keys;
+        if (tid < G) sh->cnt[tid] = sh->kk[tid] > 0 ? first_keys : 0;
       }
       // the first cut sets a useful threshold; later cuts keep room for the
       // next stretch of keys
-      check_lists<G>(buf, cap, k, t < C::SUB_ST ? k : later_limit, sh, warp,
-                     lane);
+      check_lists<G>(buf, cap, t < C::SUB_ST, long_chunk, sh, warp, lane);
     }
   }
-  check_lists<G>(buf, cap, k, k, sh, warp, lane);
+  check_lists<G>(buf, cap, true, long_chunk, sh, warp, lane);
+  if constexpr (MASS) {
+    // lanes of one head (the same l8 in each key slot ks) combine, then the
+    // warps
+#pragma unroll
+    for (int off = 8; off <= 16; off <<= 1) {
+      const float m2 = __shfl_xor_sync(0xFFFFFFFFu, ml.m, off);
+      const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ml.l, off);
+      ml.merge(m2, l2);
+    }
+    if (owner && ks == 0) sh->ml[warp][myh] = make_float2(ml.m, ml.l);
+    ComputeBar::sync();
+    if (tid < G) {
+      Lse2 c;
+      for (int w = 0; w < kComputeWarps; ++w)
+        c.merge(sh->ml[w][tid].x, sh->ml[w][tid].y);
+      const size_t lst =
+          ((size_t)b * a.Hq + (size_t)g * G + tid) * a.nchunks + chunk;
+      a.cand_ml[lst] = make_float2(c.m, c.l);
+    }
+  }
 
   // write this chunk's best keys per q-head; empty slots get key 0
 #pragma unroll 1
@@ -466,19 +517,23 @@ decode_merge_attend(DecodeArgs a) {
   float* tops = reinterpret_cast<float*>(topj + a.kpow2);       // [kpow2]
   SelectState<1>* st = reinterpret_cast<SelectState<1>*>(tops + a.kpow2);
   __shared__ int s_n, s_kk, s_m;
-  __shared__ uint64_t s_T;
+  __shared__ uint64_t s_T, s_t0[8];
   __shared__ float s_mw[NW], s_lw[NW];
   __shared__ float s_ow[NW][D];
+  __shared__ float s_wm[8], s_wl[8], s_s0;  // window+anchor states; anchor score
 
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int gtid = tid & 255, gw = warp & 7;
   const int g = h / (a.Hq / a.Hkv);
   const int64_t L = a.L, i = L - 1;
-  const int Wb = row_window(a.W_i, b, a.W, (int)L, a.status, false);
+  const int Wb = row_window(a.W_i, b, a.W_h, h, a.W, (int)L, a.status,
+                            tid == 0);
+  const int kh = head_k(a.k_h, h, k, a.status, tid == 0);
+  const bool want_mass = a.mass != nullptr || a.lse != nullptr;
   const int64_t lo = (i - Wb + 1) > 0 ? (i - Wb + 1) : 0;
   const int64_t ncand_pos = (i - Wb) > 0 ? (i - Wb) : 0;  // |[1, i-W]|
-  const int m = (int)(k < ncand_pos ? k : ncand_pos);
+  const int m = (int)(kh < ncand_pos ? kh : ncand_pos);
   const int anc = lo > 0 ? 1 : 0;
   const int64_t count = anc + m + (i - lo + 1);
 
@@ -518,21 +573,66 @@ decode_merge_attend(DecodeArgs a) {
         acc.add(dot * sl2, vf[u]);
       }
     }
+    if (want_mass) {
+      // the window + anchor part alone, and the anchor's own score (inside
+      // the window when the window reaches position 0)
+      if (lane == 0) {
+        s_wm[gw] = acc.m;
+        s_wl[gw] = acc.l;
+      }
+      if (gw == 0) {
+        float k0[DL];
+        load_f32<T, DL>(Kg, k0);
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) dot = fmaf(qv[e], k0[e], dot);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
+        if (lane == 0) s_s0 = dot * sl2;
+      }
+    }
   } else {
     // ---------------- merge the chunk lists into the exact Top-k
     // The lists are written by the score kernel, which may still be
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
+    // Every chunk list holds its chunk's best k keys, so the largest of the
+    // lists' smallest keys, T0, is at most the global k-th best key (the
+    // chunk that has it alone holds k keys >= T0): only keys >= T0 can be
+    // selected.  A list of a chunk with fewer than k candidates has empty
+    // (0) slots and contributes 0.
+    uint64_t t0 = 0ull;
+    for (int c = gw; c < a.nchunks; c += 8) {
+      uint64_t mn = ~0ull;
+      for (int e = lane; e < kh; e += 32) mn = min(mn, src[(size_t)c * k + e]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+      t0 = max(t0, mn);
+    }
+    if (lane == 0) s_t0[gw] = t0;
     if (gtid == 0) {
-      s_n = ncand;
+      s_n = 0;
       s_m = 0;
       s_kk = m > 0 ? m : 1;
     }
-    // The lists are copied as they are: empty slots (key 0) sort below every
-    // real key, and the lists hold at least m real keys, so the m-th largest
-    // key is a real one.
-    const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
-    for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
+    MergeBar::sync();
+    t0 = s_t0[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) t0 = max(t0, s_t0[w]);
+    // keep the keys >= T0 (and real), packed to the front in any order
+    for (int e0 = 0; e0 < ncand; e0 += 256) {
+      const int e = e0 + gtid;
+      const uint64_t key = e < ncand ? src[e] : 0ull;
+      const bool keep = key != 0ull && key >= t0;
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+      int base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&s_n, __popc(bal));
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
+      if (keep) cand[base + __popc(bal & ((1u << lane) - 1u))] = key;
+    }
     MergeBar::sync();
     cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
                                             gtid);
@@ -596,6 +696,18 @@ decode_merge_attend(DecodeArgs a) {
     TO* out = reinterpret_cast<TO*>(a.O) + ((size_t)b * a.Hq + h) * D;
     store_out<TO>(out + dd, o / l);
   }
+  if (want_mass && tid == 32 + D) {
+    // masses over the full causal softmax: C (all warps), window + anchor
+    // (warps 8..15 before the Top-k rows), and every candidate (the score
+    // pass's per-chunk sums), in one frame
+    Lse2 c, wa, cand;
+    for (int w = 0; w < NW; ++w) c.merge(s_mw[w], s_lw[w]);
+    for (int w = 0; w < 8; ++w) wa.merge(s_wm[w], s_wl[w]);
+    const float2* cml = a.cand_ml + ((size_t)b * a.Hq + h) * a.nchunks;
+    for (int ch = 0; ch < a.nchunks; ++ch) cand.merge(cml[ch].x, cml[ch].y);
+    mass_report(a.mass, a.lse, (size_t)b * a.Hq + h, c.m, c.l, wa.m, wa.l,
+                cand.m, cand.l, s_s0, anc != 0);
+  }
   __syncthreads();  // the sorted Top-k is visible
   int32_t* idx_row = a.idx + ((size_t)b * a.Hq + h) * a.C_max;
   if (count > a.C_max && tid == 0) raise_flag(a.status, kErrCmax);
@@ -644,8 +756,12 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   size_t smem1;
   score_smem<T, D, G>(a.k, &a.cap, &a.nstages, &smem1);
   cudaError_t e = cudaSuccess;
-  if (a.k > 0) {  // with k = 0 the set is anchor and window only
-      auto k1 = decode_score_topk<T, D, G>;
+  const bool mass = a.mass != nullptr || a.lse != nullptr;
+  // with k = 0 the set is anchor and window only: the score pass runs only
+  // for the mass reports (the candidates' sums)
+  if (a.k > 0 || mass) {
+    auto k1 = mass ? decode_score_topk<T, D, G, true>
+                   : decode_score_topk<T, D, G, false>;
     // the largest shared-memory carve-out, so that two CTAs fit per SM
     e = ensure_smem(k1, smem1, true);
     if (e != cudaSuccess) return e;

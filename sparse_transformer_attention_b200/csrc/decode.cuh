@@ -21,7 +21,13 @@ struct DecodeArgs {
   const void* K;
   const void* V;
   int B, L, Hq, Hkv, W, k;
-  const int32_t* W_i;
+  const int32_t* W_i;   // [B] or NULL
+  const int32_t* W_h;   // [Hq] or NULL
+  const int32_t* k_h;   // [Hq] or NULL
+  float* mass;          // [B*Hq, 4] or NULL
+  float* lse;           // [B*Hq] or NULL
+  float2* cand_ml;      // [B, Hq, nchunks] log2-domain (max, sum) of each
+                        // chunk's candidates, when mass or lse is asked
   void* O;
   int o_bf16;
   int32_t* idx;

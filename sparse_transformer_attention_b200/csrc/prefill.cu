@@ -39,20 +39,21 @@ namespace ca {
 namespace {
 
 // ------------------------------------------------------------ shared prologue
-// Window and last candidate position of each row of the tile; returns the
-// largest last-candidate position over the tile's rows (-1 if none).
-__device__ void tile_rows(const PrefillArgs& a, int b, int i0, int* s_hi,
-                          int* s_maxhi) {
+// Window and last candidate position of each row of the tile (query rows
+// r0 .. r0+127 of head h, at positions p0 + r); returns the largest
+// last-candidate position over the tile's rows (-1 if none).
+__device__ void tile_rows(const PrefillArgs& a, int b, int h, int r0,
+                          int* s_hi, int* s_maxhi) {
   const int tid = threadIdx.x;
   if (tid == 0) *s_maxhi = -1;
   __syncthreads();
   if (tid < kTileRows) {
-    const int i = i0 + tid;
+    const int r = r0 + tid;
     int hi = -1;
-    if (i < a.n) {
-      const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n,
-                               a.status, true);
-      hi = i - w;
+    if (r < a.nq) {
+      const int w = row_window(a.W_i, (int64_t)b * a.nq + r, a.W_h, h, a.W,
+                               a.L, a.status, true);
+      hi = a.p0 + r - w;
     }
     s_hi[tid] = hi;
     atomicMax(s_maxhi, hi);
@@ -120,6 +121,8 @@ struct TcShared {
   int maxhi;
   int hi[kTileRows];
   float L[kTileRows];
+  float M[kTileRows];       // row maximum over the candidates (mass reports)
+  float xsum[kSelThreads];  // per thread: sum of 2^((s - M) log2e/sqrt(d))
   short cnt[kSelThreads];   // entries in the thread's own segment, -1: overflow
   short xcnt[kSelThreads];  // entries in its spare segment
   signed char xcol[kSelThreads];  // spare segment index, -1: none
@@ -247,8 +250,8 @@ template <int NE>
 __device__ __forceinline__ void quad_select(const unsigned char* seg,
                                             const unsigned char* codes,
                                             const RowSegs& rs, bool live,
-                                            uint32_t lob, int k, uint64_t* out,
-                                            int part) {
+                                            uint32_t lob, int k, int kpad,
+                                            uint64_t* out, int part) {
   uint32_t hv[NE];
 #pragma unroll
   for (int t = 0; t < NE; ++t) {
@@ -354,11 +357,11 @@ __device__ __forceinline__ void quad_select(const unsigned char* seg,
         }
       }
     }
-    for (int e = total + part; e < k; e += 4) out[e] = 0ull;
+    for (int e = total + part; e < kpad; e += 4) out[e] = 0ull;
   }
 }
 
-template <int D>
+template <int D, bool MASS>
 __global__ void __launch_bounds__(kTcThreads, 1)
 prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
@@ -377,11 +380,11 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (a.Hq / a.Hkv);
-  const int i0 = qt * Lay::BM;
+  const int i0 = qt * Lay::BM;  // first query row of the tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int k = a.k;
+  const int k = head_k(a.k_h, h, a.k, a.status, qt == 0 && tid == 0);
 
-  tile_rows(a, b, i0, sh.hi, &sh.maxhi);
+  tile_rows(a, b, h, i0, sh.hi, &sh.maxhi);
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       sm100::mbar_init(&sh.kfull[s], 1);
@@ -415,8 +418,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     if (lane == 0 && T > 0) {
       sm100::prefetch_tmap(&tmQ);
       sm100::prefetch_tmap(&tmK);
-      const int qrow = ((b * a.Hq + h) * a.n) + i0;
-      const int krow = (b * a.Hkv + g) * a.n;
+      const int qrow = ((b * a.Hq + h) * a.nq) + i0;
+      const int krow = (b * a.Hkv + g) * a.L;
       sm100::mbar_arrive_expect_tx(&sh.qfull, Lay::kQBytes);
       for (int kb = 0; kb < KB; ++kb)
         sm100::tma_load_2d(sQ + kb * Lay::kBlockBytes, &tmQ, &sh.qfull, kb * 64,
@@ -585,10 +588,23 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         if (__all_sync(0xFFFFFFFFu, done)) break;
       }
       if (part == 0)
-        sh.L[row] = (tau <= ord_f32(-INFINITY)) ? -INFINITY : unord_f32(tau);
+        sh.L[row] = k == 0 ? INFINITY  // nothing to select: no appends
+                    : (tau <= ord_f32(-INFINITY)) ? -INFINITY
+                                                  : unord_f32(tau);
+      if constexpr (MASS) {
+        uint32_t mx = 0u;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) mx = max(mx, key[x]);
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+        if (part == 0) sh.M[row] = unord_f32(mx);
+      }
     }
     SelBar::sync();
     const float Lr = sh.L[r];
+    const float sl2 = 1.4426950408889634f / sqrtf((float)D);
+    const float Mr = MASS ? sh.M[r] : 0.f;
+    float xs = 0.f;  // this thread's share of the candidates' sum
     // ---- pass 2: append every candidate >= L to this thread's segment; a
     // full segment continues in a spare one (rare), else the row is listed
     // for the exact fallback.
@@ -609,6 +625,11 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int x = 0; x < 32; ++x)
           if (!(j0 + x >= 1 && j0 + x <= hi)) raw[x] = kMaskedScore;
+      }
+      if constexpr (MASS) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          xs += exp2f(fmaxf((__uint_as_float(raw[x]) - Mr) * sl2, -INFINITY));
       }
       const uint32_t cbase = (uint32_t)tile * 32;
       const uint32_t as_t = as;  // cursor at the tile start
@@ -645,15 +666,16 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sh.cnt[col] = ovf ? (short)-1 : (short)(xc < 0 ? last : own);
     sh.xcnt[col] = (short)(xc < 0 ? 0 : last);
     sh.xcol[col] = (signed char)xc;
+    if constexpr (MASS) sh.xsum[col] = xs;
     SelBar::sync();
     // ---- exact Top-k per row: four lanes per row, eight rows per warp
     {
       const int row = sw * 8 + (lane >> 2), part = lane & 3;
-      const int i = i0 + row;
+      const int r = i0 + row;
       RowSegs rs;
       row_segs(sh, row, rs);
-      const size_t grow = (size_t)(b * a.Hq + h) * a.n + i;
-      bool live = i < a.n;
+      const size_t grow = (size_t)(b * a.Hq + h) * a.nq + r;
+      bool live = r < a.nq;
       if (live && (rs.bad || rs.n > 128)) {
         // listed for the exact fallback pass; it writes this row
         if (part == 0) {
@@ -662,12 +684,19 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         }
         live = false;
       }
+      if constexpr (MASS) {
+        float t = sh.xsum[part * kTileRows + row];
+        t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
+        t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
+        if (r < a.nq && part == 0)
+          a.cand_ml[grow] = make_float2(sh.M[row] * sl2, t);
+      }
       const uint32_t lob = ord_f32(sh.L[row]);
-      uint64_t* out = a.topk + grow * k;
+      uint64_t* out = a.topk + grow * a.k;
       if (__all_sync(0xFFFFFFFFu, !live || rs.n <= 64))
-        quad_select<16>(seg, codes, rs, live, lob, k, out, part);
+        quad_select<16>(seg, codes, rs, live, lob, k, a.k, out, part);
       else
-        quad_select<32>(seg, codes, rs, live, lob, k, out, part);
+        quad_select<32>(seg, codes, rs, live, lob, k, a.k, out, part);
     }
   }
   __syncwarp();  // reconverge single-lane roles before the CTA barrier
@@ -739,15 +768,17 @@ prefill_overflow_rows(PrefillArgs a) {
   const uint32_t nrows = *a.ovf_count;
   for (uint32_t it = blockIdx.x; it < nrows; it += gridDim.x) {
     const uint32_t grow = a.ovf_rows[it];
-    const int i = (int)(grow % (uint32_t)a.n);
-    const uint32_t bh = grow / (uint32_t)a.n;
+    const int r = (int)(grow % (uint32_t)a.nq);
+    const uint32_t bh = grow / (uint32_t)a.nq;
     const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
     const int g = h / (a.Hq / a.Hkv);
-    const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n, a.status,
-                             false);
-    const int hi = i - w;
+    const int w = row_window(a.W_i, (int64_t)b * a.nq + r, a.W_h, h, a.W,
+                             a.L, a.status, false);
+    const int kh = head_k(a.k_h, h, k, a.status, false);
+    const int hi = a.p0 + r - w;
     const T* Qr = reinterpret_cast<const T*>(a.Q) + (size_t)grow * D;
-    const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * a.n * D;
+    const T* Kg = reinterpret_cast<const T*>(a.K) +
+                  ((size_t)b * a.Hkv + g) * (size_t)a.L * D;
     for (int e = threadIdx.x; e < D; e += kFbThreads) q[e] = Elem<T>::load1(Qr + e);
     if (threadIdx.x == 0) {
       s_n = 0;
@@ -782,8 +813,8 @@ prefill_overflow_rows(PrefillArgs a) {
       }
       __syncthreads();
       const bool last = c0 + kFbChunk > hi;
-      if (last ? s_n > k : s_n > k + kFbBuf - kFbChunk) {  // uniform
-        if (threadIdx.x == 0) s_kk = k;
+      if (last ? s_n > kh : s_n > k + kFbBuf - kFbChunk) {  // uniform
+        if (threadIdx.x == 0) s_kk = kh;
         __syncthreads();
         cta_select_thresholds<kFbThreads, 1>(keys, 0, &s_n, &s_kk, &s_T, &st,
                                              threadIdx.x);
@@ -797,7 +828,7 @@ prefill_overflow_rows(PrefillArgs a) {
         for (int c = 0; c < cntm; ++c)
           if (mine[c] >= s_T) keys[atomicAdd(&s_w, 1)] = mine[c];
         __syncthreads();
-        if (threadIdx.x == 0) s_n = k;
+        if (threadIdx.x == 0) s_n = kh;
         __syncthreads();
       }
     }
@@ -808,7 +839,7 @@ prefill_overflow_rows(PrefillArgs a) {
 }
 
 // ============================================================ fp32 FFMA kernel
-template <int D>
+template <int D, bool MASS>
 __global__ void __launch_bounds__(kTileRows)
 prefill_score_topk_f32(PrefillArgs a) {
   constexpr int TJ = 32;     // keys per tile
@@ -822,31 +853,34 @@ prefill_score_topk_f32(PrefillArgs a) {
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (a.Hq / a.Hkv);
-  const int i0 = qt * kTileRows;
-  const int r = threadIdx.x, i = i0 + r;
-  tile_rows(a, b, i0, s_hi, &s_maxhi);
+  const int i0 = qt * kTileRows;  // first query row of the tile
+  const int r = threadIdx.x, row = i0 + r;
+  const int kh = head_k(a.k_h, h, a.k, a.status, qt == 0 && r == 0);
+  tile_rows(a, b, h, i0, s_hi, &s_maxhi);
   const int hi = s_hi[r];
   const int maxhi = s_maxhi;
 
   float q[D];
   const float* Qr = reinterpret_cast<const float*>(a.Q) +
-                    ((size_t)(b * a.Hq + h) * a.n + (i < a.n ? i : 0)) * D;
+                    ((size_t)(b * a.Hq + h) * a.nq + (row < a.nq ? row : 0)) * D;
 #pragma unroll
   for (int e = 0; e < D; e += 4) {
     float4 v = *reinterpret_cast<const float4*>(Qr + e);
     q[e] = v.x; q[e + 1] = v.y; q[e + 2] = v.z; q[e + 3] = v.w;
   }
   const float* Kg = reinterpret_cast<const float*>(a.K) +
-                    (size_t)(b * a.Hkv + g) * a.n * D;
+                    (size_t)(b * a.Hkv + g) * a.L * D;
+  const float sl2 = 1.4426950408889634f / sqrtf((float)D);
+  float mrow = -INFINITY, lrow = 0.f;  // candidates' (max, sum) for masses
   RowTopk sel;
-  sel.init(heap, stage, r, a.k, S);
+  sel.init(heap, stage, r, kh, S);
   const int T = maxhi >= 1 ? maxhi / TJ + 1 : 0;
   for (int t = 0; t < T; ++t) {
     __syncthreads();
     for (int e = threadIdx.x * 4; e < TJ * D; e += kTileRows * 4) {
       const int jj = t * TJ + e / D;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (jj < a.n) v = *reinterpret_cast<const float4*>(Kg + (size_t)jj * D + e % D);
+      if (jj < a.L) v = *reinterpret_cast<const float4*>(Kg + (size_t)jj * D + e % D);
       *reinterpret_cast<float4*>(sK + e) = v;
     }
     __syncthreads();
@@ -865,15 +899,40 @@ prefill_score_topk_f32(PrefillArgs a) {
       raw[c] = __float_as_uint(acc);
     }
     const int j0 = t * TJ;
-    const bool interior = (j0 >= 1) && (j0 + 31 <= hi);
-    if (__all_sync(0xFFFFFFFFu, interior))
-      sel.offer<false>(raw, j0, 1, hi);
-    else
-      sel.offer<true>(raw, j0, 1, hi);
+    if constexpr (MASS) {
+      float tm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < TJ; ++c)
+        if (j0 + c >= 1 && j0 + c <= hi)
+          tm = fmaxf(tm, __uint_as_float(raw[c]));
+      if (tm > -INFINITY) {
+        const float mn = fmaxf(mrow, tm);
+        lrow *= exp2f((mrow - mn) * sl2);
+#pragma unroll
+        for (int c = 0; c < TJ; ++c)
+          if (j0 + c >= 1 && j0 + c <= hi)
+            lrow += exp2f((__uint_as_float(raw[c]) - mn) * sl2);
+        mrow = mn;
+      }
+    }
+    if (kh > 0) {  // uniform over the CTA (one head)
+      const bool interior = (j0 >= 1) && (j0 + 31 <= hi);
+      if (__all_sync(0xFFFFFFFFu, interior))
+        sel.offer<false>(raw, j0, 1, hi);
+      else
+        sel.offer<true>(raw, j0, 1, hi);
+    }
   }
-  sel.drain();
-  if (i < a.n && a.k > 0)
-    sel.store(a.topk + ((size_t)(b * a.Hq + h) * a.n + i) * a.k);
+  const size_t grow = (size_t)(b * a.Hq + h) * a.nq + row;
+  if (kh > 0) sel.drain();
+  if (row < a.nq && a.k > 0) {
+    uint64_t* out = a.topk + grow * a.k;
+    sel.store(out);
+    for (int e = kh; e < a.k; ++e) out[e] = 0ull;
+  }
+  if constexpr (MASS) {
+    if (row < a.nq) a.cand_ml[grow] = make_float2(mrow * sl2, lrow);
+  }
 }
 
 // ============================================================ gather kernel
@@ -917,14 +976,50 @@ constexpr int kGatherWarps = 8;
 constexpr int kGatherRPW = 4;              // rows per warp
 constexpr int kGatherLPR = 32 / kGatherRPW;  // lanes per row
 
-template <typename T, int D, typename TO, int NPL>
+// Write C_i (ascending, -1 padded) and |C_i| of one row, with the whole
+// warp: v[] holds the row's Top-k positions (0xFFFFFFFF for empty slots,
+// element t*32 + lane in v[t]), m of them real.
+template <int NPL>
+__device__ __forceinline__ void write_set(const PrefillArgs& a, int64_t row,
+                                          uint32_t (&v)[NPL], int m, int i,
+                                          int lo, int lane) {
+  warp_sort<NPL>(v, lane);
+  const int anc = lo > 0 ? 1 : 0;
+  const int count = anc + m + (i - lo + 1);
+  if (count > a.C_max && lane == 0) raise_flag(a.status, kErrCmax);
+  const int wcount = count < a.C_max ? count : a.C_max;
+  int32_t* out = a.idx + row * a.C_max;
+  for (int rb = 0; rb < a.C_max; rb += 32) {
+    const int rpos = rb + lane;
+    // the sorted Top-k value for slot rpos-anc sits in lane (rpos-anc)%32
+    const int tk = rpos - anc;
+    uint32_t sv = 0;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      const uint32_t x = __shfl_sync(0xFFFFFFFFu, v[t], tk & 31);
+      if ((tk >> 5) == t) sv = x;
+    }
+    if (rpos < a.C_max) {
+      int32_t val;
+      if (rpos >= wcount) val = -1;
+      else if (rpos < anc) val = 0;
+      else if (tk < m) val = (int32_t)sv;
+      else val = lo + (tk - m);
+      out[rpos] = val;
+    }
+  }
+  if (lane == 0) a.idx_count[row] = count;
+}
+
+template <typename T, int D, typename TO, int NPL, bool MASS>
 __global__ void __launch_bounds__(kGatherWarps * 32)
 prefill_gather(PrefillArgs a) {
   constexpr int DL = D / kGatherLPR;
   constexpr int KPC = 4;  // keys per chunk
   __shared__ uint64_t s_key[kGatherWarps][kGatherRPW][kPrefillMaxK];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t R = (int64_t)a.B * a.Hq * a.n;
+  const int nq = a.nq;
+  const int64_t R = (int64_t)a.B * a.Hq * nq;
   const int64_t row0 = ((int64_t)blockIdx.x * kGatherWarps + wid) * kGatherRPW;
   if (row0 >= R) return;  // the whole warp
   const int k = a.k;
@@ -934,13 +1029,13 @@ prefill_gather(PrefillArgs a) {
   for (int rr = 0; rr < kGatherRPW; ++rr) {
     const int64_t row = row0 + rr;
     if (row >= R) break;
-    const int64_t bh = row / a.n;
-    const int i = (int)(row - bh * a.n);
-    const int b = (int)(bh / a.Hq);
-    const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n, a.status,
-                             false);
+    const int64_t bh = row / nq;
+    const int r = (int)(row - bh * nq);
+    const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
+    const int i = a.p0 + r;
+    const int w = row_window(a.W_i, (int64_t)b * nq + r, a.W_h, h, a.W, a.L,
+                             a.status, false);
     const int lo = i - w + 1 > 0 ? i - w + 1 : 0;
-    const int anc = lo > 0 ? 1 : 0;
     uint32_t v[NPL];
     int m = 0;
 #pragma unroll
@@ -952,31 +1047,7 @@ prefill_gather(PrefillArgs a) {
       v[t] = key ? key_index(key) : 0xFFFFFFFFu;
       m += __popc(__ballot_sync(0xFFFFFFFFu, key != 0ull));
     }
-    warp_sort<NPL>(v, lane);
-    const int count = anc + m + (i - lo + 1);
-    if (count > a.C_max && lane == 0) raise_flag(a.status, kErrCmax);
-    const int wcount = count < a.C_max ? count : a.C_max;
-    int32_t* out = a.idx + row * a.C_max;
-    for (int rb = 0; rb < a.C_max; rb += 32) {
-      const int rpos = rb + lane;
-      // the sorted Top-k value for slot rpos-anc sits in lane (rpos-anc)%32
-      const int tk = rpos - anc;
-      uint32_t sv = 0;
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) {
-        const uint32_t x = __shfl_sync(0xFFFFFFFFu, v[t], tk & 31);
-        if ((tk >> 5) == t) sv = x;
-      }
-      if (rpos < a.C_max) {
-        int32_t val;
-        if (rpos >= wcount) val = -1;
-        else if (rpos < anc) val = 0;
-        else if (tk < m) val = (int32_t)sv;
-        else val = lo + (tk - m);
-        out[rpos] = val;
-      }
-    }
-    if (lane == 0) a.idx_count[row] = count;
+    write_set<NPL>(a, row, v, m, i, lo, lane);
   }
   __syncwarp();
 
@@ -985,18 +1056,19 @@ prefill_gather(PrefillArgs a) {
   const int64_t row = row0 + rloc;
   const bool live = row < R;
   const int64_t rowc = live ? row : R - 1;
-  const int64_t bh = rowc / a.n;
-  const int i = (int)(rowc - bh * a.n);
+  const int64_t bh = rowc / nq;
+  const int r = (int)(rowc - bh * nq);
   const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
   const int g = h / (a.Hq / a.Hkv);
-  const int w = row_window(a.W_i, (int64_t)b * a.n + i, a.W, a.n, a.status,
-                           false);
+  const int i = a.p0 + r;
+  const int w = row_window(a.W_i, (int64_t)b * nq + r, a.W_h, h, a.W, a.L,
+                           a.status, false);
   const int lo = i - w + 1 > 0 ? i - w + 1 : 0;
   const int anc = lo > 0 ? 1 : 0;
   const T* Kg = reinterpret_cast<const T*>(a.K) +
-                ((size_t)b * a.Hkv + g) * a.n * D + sub * DL;
+                ((size_t)b * a.Hkv + g) * (size_t)a.L * D + sub * DL;
   const T* Vg = reinterpret_cast<const T*>(a.V) +
-                ((size_t)b * a.Hkv + g) * a.n * D + sub * DL;
+                ((size_t)b * a.Hkv + g) * (size_t)a.L * D + sub * DL;
   float qv[DL];
   {
     RawRow<T, DL> qr;
@@ -1031,27 +1103,7 @@ prefill_gather(PrefillArgs a) {
     mrun = mn;
   };
 
-  // Top-k entries: the selector's fp32 scores
-  for (int c0 = 0; c0 < k; c0 += KPC) {
-    float s[KPC];
-    RawRow<T, DL> vr[KPC];
-#pragma unroll
-    for (int u = 0; u < KPC; ++u) {
-      const int e = c0 + u;
-      const uint64_t key = (live && e < k) ? s_key[wid][rloc][e] : 0ull;
-      uint32_t j = key ? key_index(key) : 0u;
-      bool act = key != 0ull;
-      if (act && (j == 0 || (int)j > i - w)) {  // never written by the selector
-        raise_flag(a.status, kErrInternal);
-        act = false;
-        j = 0;
-      }
-      s[u] = act ? key_score(key) * sl2 : -INFINITY;
-      vr[u].load(Vg + (size_t)j * D);
-    }
-    fold(s, vr);
-  }
-  // anchor and window: dot products over the row's eight lanes
+  // anchor and window first: dot products over the row's eight lanes
   const int nw = live ? anc + (i - lo + 1) : 0;
   int nmax = nw;
 #pragma unroll
@@ -1090,11 +1142,50 @@ prefill_gather(PrefillArgs a) {
       s[u] = (c0 + u < nw) ? s[u] * sl2 : -INFINITY;
     fold(s, vr);
   }
+  const float m_wa = mrun, l_wa = den;  // window + anchor alone
+  // Top-k entries: the selector's fp32 scores
+  for (int c0 = 0; c0 < k; c0 += KPC) {
+    float s[KPC];
+    RawRow<T, DL> vr[KPC];
+#pragma unroll
+    for (int u = 0; u < KPC; ++u) {
+      const int e = c0 + u;
+      const uint64_t key = (live && e < k) ? s_key[wid][rloc][e] : 0ull;
+      uint32_t j = key ? key_index(key) : 0u;
+      bool act = key != 0ull;
+      if (act && (j == 0 || (int64_t)j > (int64_t)(i - w))) {  // not a candidate
+        raise_flag(a.status, kErrInternal);
+        act = false;
+        j = 0;
+      }
+      s[u] = act ? key_score(key) * sl2 : -INFINITY;
+      vr[u].load(Vg + (size_t)j * D);
+    }
+    fold(s, vr);
+  }
   if (live) {
     TO* op = reinterpret_cast<TO*>(a.O) + rowc * D + sub * DL;
     const float inv = 1.f / den;
 #pragma unroll
     for (int e = 0; e < DL; ++e) store_out<TO>(op + e, o[e] * inv);
+  }
+  if constexpr (MASS) {
+    // the anchor's own score (inside the window when it reaches 0)
+    RawRow<T, DL> k0;
+    k0.load(Kg);
+    float kf[DL];
+    k0.to_f32(kf);
+    float d0 = 0.f;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) d0 = fmaf(qv[e], kf[e], d0);
+#pragma unroll
+    for (int off = kGatherLPR / 2; off > 0; off >>= 1)
+      d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, off);
+    if (live && sub == 0) {
+      const float2 cm = a.cand_ml[row];
+      mass_report(a.mass, a.lse, (size_t)row, mrun, den, m_wa, l_wa, cm.x,
+                  cm.y, d0 * sl2, anc != 0);
+    }
   }
 }
 
@@ -1158,7 +1249,7 @@ struct MmaGatherSmem {
 //   3. Eight lanes per row, four rows at a time: start from the window state
 //      and fold in the Top-k keys (scores from the selector) and the anchor
 //      (score computed here), then write the output row.
-template <int D, typename TO, int NPL>
+template <int D, typename TO, int NPL, bool MASS>
 __global__ void __launch_bounds__(kMmaWarps * 32)
 prefill_gather_mma(PrefillArgs a) {
   using T = __nv_bfloat16;
@@ -1166,7 +1257,8 @@ prefill_gather_mma(PrefillArgs a) {
   constexpr int NT = D / 8;   // head-dim tiles of the p * V MMA
   extern __shared__ __align__(16) unsigned char g_smem[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int n = a.n, k = a.k;
+  // query rows r at positions p0 + r, keys 0..L-1
+  const int nq = a.nq, L = a.L, p0 = a.p0, k = a.k;
   float* s_o = reinterpret_cast<float*>(g_smem + wid * MmaGatherSmem<D>::per_warp(k));
   float* s_m = s_o + 16 * D;
   float* s_l = s_m + 16;
@@ -1174,18 +1266,18 @@ prefill_gather_mma(PrefillArgs a) {
   const int bh = blockIdx.y;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const int i0 = (blockIdx.x * kMmaWarps + wid) * 16;
-  if (i0 >= n) return;  // the whole warp
-  const int64_t rowbase = (int64_t)bh * n;
+  const int i0 = (blockIdx.x * kMmaWarps + wid) * 16;  // first query row
+  if (i0 >= nq) return;  // the whole warp
+  const int64_t rowbase = (int64_t)bh * nq;
   const T* Qg = reinterpret_cast<const T*>(a.Q) + rowbase * D;
-  const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * n * D;
-  const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * n * D;
+  const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * (size_t)L * D;
+  const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * (size_t)L * D;
 
   // ---- 1: the Top-k keys of the warp's rows (16 consecutive rows of one
   // head: one contiguous run) into shared memory, 16 loads in flight per
   // lane, then C_i one row at a time across the warp
   {
-    const int nk = min(16, n - i0) * k;
+    const int nk = min(16, nq - i0) * k;
     const uint64_t* kg = a.topk + (rowbase + i0) * k;
 #pragma unroll 1
     for (int e0 = 0; e0 < nk; e0 += 16 * 32) {
@@ -1205,12 +1297,12 @@ prefill_gather_mma(PrefillArgs a) {
   }
 #pragma unroll 1
   for (int rr = 0; rr < 16; ++rr) {
-    const int i = i0 + rr;
-    if (i >= n) break;
-    const int64_t row = rowbase + i;
-    const int w = row_window(a.W_i, (int64_t)b * n + i, a.W, n, a.status, false);
+    const int r = i0 + rr;
+    if (r >= nq) break;
+    const int i = p0 + r;  // position
+    const int w = row_window(a.W_i, (int64_t)b * nq + r, a.W_h, h, a.W, L,
+                             a.status, false);
     const int lo = i - w + 1 > 0 ? i - w + 1 : 0;
-    const int anc = lo > 0 ? 1 : 0;
     uint32_t v[NPL];
     int m = 0;
 #pragma unroll
@@ -1220,47 +1312,27 @@ prefill_gather_mma(PrefillArgs a) {
       v[t] = key ? key_index(key) : 0xFFFFFFFFu;
       m += __popc(__ballot_sync(0xFFFFFFFFu, key != 0ull));
     }
-    warp_sort<NPL>(v, lane);
-    const int count = anc + m + (i - lo + 1);
-    if (count > a.C_max && lane == 0) raise_flag(a.status, kErrCmax);
-    const int wcount = count < a.C_max ? count : a.C_max;
-    int32_t* out = a.idx + row * a.C_max;
-    for (int rb = 0; rb < a.C_max; rb += 32) {
-      const int rpos = rb + lane;
-      const int tk = rpos - anc;
-      uint32_t sv = 0;
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) {
-        const uint32_t x = __shfl_sync(0xFFFFFFFFu, v[t], tk & 31);
-        if ((tk >> 5) == t) sv = x;
-      }
-      if (rpos < a.C_max) {
-        int32_t val;
-        if (rpos >= wcount) val = -1;
-        else if (rpos < anc) val = 0;
-        else if (tk < m) val = (int32_t)sv;
-        else val = lo + (tk - m);
-        out[rpos] = val;
-      }
-    }
-    if (lane == 0) a.idx_count[row] = count;
+    write_set<NPL>(a, rowbase + r, v, m, i, lo, lane);
   }
 
   // ---- 2: window on tensor cores
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);
   const int gr = lane >> 2, tq = lane & 3;  // fragment row group, thread in group
-  const int ia = i0 + gr, ib = i0 + gr + 8;  // this lane's two rows
-  const bool va = ia < n, vb = ib < n;
-  const int ca = va ? ia : n - 1, cb = vb ? ib : n - 1;
-  const int wa = row_window(a.W_i, (int64_t)b * n + ca, a.W, n, a.status, false);
-  const int wb = row_window(a.W_i, (int64_t)b * n + cb, a.W, n, a.status, false);
-  const int loa = ca - wa + 1 > 0 ? ca - wa + 1 : 0;
-  const int lob = cb - wb + 1 > 0 ? cb - wb + 1 : 0;
+  const int ra = i0 + gr, rb = i0 + gr + 8;  // this lane's two rows
+  const bool va = ra < nq, vb = rb < nq;
+  const int ca = va ? ra : nq - 1, cb = vb ? rb : nq - 1;
+  const int ia = p0 + ca, ib = p0 + cb;      // their positions
+  const int wa = row_window(a.W_i, (int64_t)b * nq + ca, a.W_h, h, a.W, L,
+                            a.status, false);
+  const int wb = row_window(a.W_i, (int64_t)b * nq + cb, a.W_h, h, a.W, L,
+                            a.status, false);
+  const int loa = ia - wa + 1 > 0 ? ia - wa + 1 : 0;
+  const int lob = ib - wb + 1 > 0 ? ib - wb + 1 : 0;
   int kmin = min(loa, lob);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1)
     kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, off));
-  const int kmax = min(i0 + 15, n - 1);
+  const int kmax = p0 + min(i0 + 15, nq - 1);
   uint32_t qa[KS][4];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
@@ -1281,7 +1353,7 @@ prefill_gather_mma(PrefillArgs a) {
 #pragma unroll
     for (int h8 = 0; h8 < 2; ++h8) {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int krow = min(j0 + 8 * h8 + gr, n - 1);
+      const int krow = min(j0 + 8 * h8 + gr, L - 1);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         const int c = 16 * ks + 2 * tq;
@@ -1331,8 +1403,8 @@ prefill_gather_mma(PrefillArgs a) {
     // score fragment is the A fragment as it stands
 #pragma unroll
     for (int h8 = 0; h8 < 2; ++h8) {
-      const int kv0 = min(j0 + 8 * h8 + 2 * tq, n - 1);
-      const int kv1 = min(j0 + 8 * h8 + 2 * tq + 1, n - 1);
+      const int kv0 = min(j0 + 8 * h8 + 2 * tq, L - 1);
+      const int kv1 = min(j0 + 8 * h8 + 2 * tq + 1, L - 1);
 #pragma unroll
       for (int nd = 0; nd < NT; ++nd) {
         const uint32_t b0 = bf16_bits_as_f32(Vg + (size_t)kv0 * D + 8 * nd + gr);
@@ -1373,19 +1445,21 @@ prefill_gather_mma(PrefillArgs a) {
 #pragma unroll 1
   for (int rg = 0; rg < 4; ++rg) {
     const int r = rg * 4 + rq;
-    const int i = i0 + r;
-    const bool live = i < n;
-    const int ic = live ? i : n - 1;
-    const int64_t row = rowbase + ic;
-    const int w = row_window(a.W_i, (int64_t)b * n + ic, a.W, n, a.status, false);
+    const bool live = i0 + r < nq;
+    const int rc = live ? i0 + r : nq - 1;  // query row (clamped)
+    const int ic = p0 + rc;                 // its position
+    const int64_t row = rowbase + rc;
+    const int w = row_window(a.W_i, (int64_t)b * nq + rc, a.W_h, h, a.W, L,
+                             a.status, false);
     const int lo = ic - w + 1 > 0 ? ic - w + 1 : 0;
+    const float m_win = s_m[r], l_win = s_l[r];  // the window alone
     float mrun = s_m[r], den = s_l[r], ov[DL];
 #pragma unroll
     for (int e = 0; e < DL; ++e) ov[e] = s_o[r * D + sub * DL + e];
     float qv[DL];
     {
       RawRow<T, DL> qr;
-      qr.load(Qg + (size_t)ic * D + sub * DL);
+      qr.load(Qg + (size_t)rc * D + sub * DL);
       qr.to_f32(qv);
     }
     auto fold = [&](const float (&sc)[KPC], const RawRow<T, DL> (&vr)[KPC]) {
@@ -1419,7 +1493,7 @@ prefill_gather_mma(PrefillArgs a) {
         const uint64_t key = (live && e < k) ? s_key[r * k + e] : 0ull;
         uint32_t j = key ? key_index(key) : 0u;
         bool act = key != 0ull;
-        if (act && (j == 0 || (int)j > ic - w)) {  // never written by the selector
+        if (act && (j == 0 || (int64_t)j > (int64_t)(ic - w))) {  // not a candidate
           raise_flag(a.status, kErrInternal);
           act = false;
           j = 0;
@@ -1450,6 +1524,16 @@ prefill_gather_mma(PrefillArgs a) {
 #pragma unroll
         for (int e = 0; e < DL; ++e) ov[e] = fmaf(pw, vf[e], ov[e] * f);
         mrun = mn;
+      }
+      if constexpr (MASS) {
+        if (live && sub == 0) {
+          Lse2 wa;  // window + anchor
+          wa.merge(m_win, l_win);
+          if (lo > 0) wa.add(d0 * sl2);
+          const float2 cm = a.cand_ml[row];
+          mass_report(a.mass, a.lse, (size_t)row, mrun, den, wa.m, wa.l, cm.x,
+                      cm.y, d0 * sl2, lo > 0);
+        }
       }
     }
     if (live) {
@@ -1492,14 +1576,18 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
+bool want_mass(const PrefillArgs& a) {
+  return a.mass != nullptr || a.lse != nullptr;
+}
+
 template <int D>
 cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   using Lay = TcLayout<D>;
   // segment codes hold tile * 32 + column in 16 bits
-  if ((a.n + Lay::BN - 1) / Lay::BN > 2048) return cudaErrorNotSupported;
+  if ((a.L + Lay::BN - 1) / Lay::BN > 2048) return cudaErrorNotSupported;
   CUtensorMap tq, tk;
-  if (!make_tmap(&tq, a.Q, (uint64_t)a.B * a.Hq * a.n, D)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tk, a.K, (uint64_t)a.B * a.Hkv * a.n, D)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tq, a.Q, (uint64_t)a.B * a.Hq * a.nq, D)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tk, a.K, (uint64_t)a.B * a.Hkv * a.L, D)) return cudaErrorInvalidValue;
   // Segment positions per (row, chunk group) thread: about k/4 entries are
   // expected (1.1-1.4 k per row), but one key tile can put 31 entries into
   // one segment (rows with fewer than k candidates); the cursor check every
@@ -1509,15 +1597,17 @@ cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
   while (P > kMinSeg && Lay::bytes(P) > budget) --P;
   if (Lay::bytes(P) > budget || P < 40) return cudaErrorNotSupported;
   const size_t smem = Lay::bytes(P);
-  auto kern = prefill_score_topk_tc<D>;
+  auto kern = want_mass(a) ? prefill_score_topk_tc<D, true>
+                           : prefill_score_topk_tc<D, false>;
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.n + 127) / 128, a.Hq, a.B);
+  dim3 grid((a.nq + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_tc");
   kern<<<grid, kTcThreads, smem, s>>>(tq, tk, a, P);
   prof_after(s);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.k == 0) return cudaSuccess;  // run for the mass reports only
   // rows whose segments overflowed (rare on typical inputs): exact fallback
   const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
   prof_before(s, "prefill_overflow_rows");
@@ -1530,44 +1620,46 @@ template <int D>
 cudaError_t launch_select_f32(const PrefillArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)32 * D * 4 + (size_t)a.k * kTileRows * 8 +
                       (size_t)32 * kTileRows * 8;
-  auto kern = prefill_score_topk_f32<D>;
+  auto kern = want_mass(a) ? prefill_score_topk_f32<D, true>
+                           : prefill_score_topk_f32<D, false>;
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.n + 127) / 128, a.Hq, a.B);
+  dim3 grid((a.nq + 127) / 128, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_f32");
   kern<<<grid, kTileRows, smem, s>>>(a);
   prof_after(s);
   return cudaGetLastError();
 }
 
+template <typename T, int D, typename TO, int NPL>
+void gather_f32_as(const PrefillArgs& a, dim3 grid, int nt, cudaStream_t s) {
+  if (want_mass(a)) prefill_gather<T, D, TO, NPL, true><<<grid, nt, 0, s>>>(a);
+  else prefill_gather<T, D, TO, NPL, false><<<grid, nt, 0, s>>>(a);
+}
+
 template <typename T, int D>
 cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
-  const int64_t R = (int64_t)a.B * a.Hq * a.n;
+  const int64_t R = (int64_t)a.B * a.Hq * a.nq;
   const int64_t rows_per_cta = (int64_t)kGatherWarps * kGatherRPW;
   dim3 grid((unsigned)((R + rows_per_cta - 1) / rows_per_cta));
   const int nt = kGatherWarps * 32;
   prof_before(s, "prefill_gather");
   if (a.k <= 32) {
-    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 1><<<grid, nt, 0, s>>>(a);
-    else prefill_gather<T, D, float, 1><<<grid, nt, 0, s>>>(a);
+    if (a.o_bf16) gather_f32_as<T, D, __nv_bfloat16, 1>(a, grid, nt, s);
+    else gather_f32_as<T, D, float, 1>(a, grid, nt, s);
   } else {
-    if (a.o_bf16) prefill_gather<T, D, __nv_bfloat16, 2><<<grid, nt, 0, s>>>(a);
-    else prefill_gather<T, D, float, 2><<<grid, nt, 0, s>>>(a);
+    if (a.o_bf16) gather_f32_as<T, D, __nv_bfloat16, 2>(a, grid, nt, s);
+    else gather_f32_as<T, D, float, 2>(a, grid, nt, s);
   }
   prof_after(s);
   return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
-  dim3 grid((unsigned)((a.n + 16 * kMmaWarps - 1) / (16 * kMmaWarps)),
-            (unsigned)(a.B * a.Hq));
-  const size_t smem = MmaGatherSmem<D>::bytes(a.k);
-  auto k1 = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, 1>
-                     : prefill_gather_mma<D, float, 1>;
-  auto k2 = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, 2>
-                     : prefill_gather_mma<D, float, 2>;
-  auto kern = a.k <= 32 ? k1 : k2;
+template <int D, int NPL, bool MASS>
+cudaError_t gather_mma_as(const PrefillArgs& a, dim3 grid, size_t smem,
+                          cudaStream_t s) {
+  auto kern = a.o_bf16 ? prefill_gather_mma<D, __nv_bfloat16, NPL, MASS>
+                       : prefill_gather_mma<D, float, NPL, MASS>;
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   prof_before(s, "prefill_gather");
@@ -1576,23 +1668,37 @@ cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
+  dim3 grid((unsigned)((a.nq + 16 * kMmaWarps - 1) / (16 * kMmaWarps)),
+            (unsigned)(a.B * a.Hq));
+  const size_t smem = MmaGatherSmem<D>::bytes(a.k);
+  const bool m = want_mass(a);
+  if (a.k <= 32)
+    return m ? gather_mma_as<D, 1, true>(a, grid, smem, s)
+             : gather_mma_as<D, 1, false>(a, grid, smem, s);
+  return m ? gather_mma_as<D, 2, true>(a, grid, smem, s)
+           : gather_mma_as<D, 2, false>(a, grid, smem, s);
+}
+
 }  // namespace
 
-size_t prefill_topk_bytes(int B, int n, int Hq, int k) {
-  size_t bytes = (size_t)B * Hq * n * (size_t)(k > 0 ? k : 1) * 8;
+size_t prefill_topk_bytes(int64_t rows, int k) {
+  size_t bytes = (size_t)rows * (size_t)(k > 0 ? k : 1) * 8;
   return (bytes + 255) / 256 * 256;
 }
 
-size_t prefill_workspace(bool, int B, int n, int Hq, int, int, int k) {
-  // per-row Top-k keys, then the list of rows for the exact fallback
-  return prefill_topk_bytes(B, n, Hq, k) +
-         ((size_t)B * Hq * n * 4 + 255) / 256 * 256;
+size_t prefill_workspace(int64_t rows, int k) {
+  // per-row Top-k keys, the list of rows for the exact fallback, and the
+  // candidates' (max, sum) per row for the mass reports
+  return prefill_topk_bytes(rows, k) + ((size_t)rows * 4 + 255) / 256 * 256 +
+         ((size_t)rows * 8 + 255) / 256 * 256;
 }
 
 cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,
                            cudaStream_t s) {
   cudaError_t e = cudaSuccess;
-  if (a.k > 0) {
+  if (a.k > 0 || want_mass(a)) {
     if (bf16) e = d == 64 ? launch_select_tc<64>(a, s) : launch_select_tc<128>(a, s);
     else e = d == 64 ? launch_select_f32<64>(a, s) : launch_select_f32<128>(a, s);
     if (e != cudaSuccess) return e;

@@ -11,11 +11,19 @@ namespace ca {
 constexpr int kPrefillMaxK = 64;
 
 struct PrefillArgs {
-  const void* Q;
-  const void* K;
+  const void* Q;   // [B, Hq, nq, d]
+  const void* K;   // [B, Hkv, L, d]
   const void* V;
-  int B, n, Hq, Hkv, W, k;
-  const int32_t* W_i;
+  // nq query rows per (batch, head) at positions p0 .. p0+nq-1 (p0 = L-nq)
+  // against L keys
+  int B, nq, L, p0, Hq, Hkv, W, k;
+  const int32_t* W_i;   // [B, nq] or NULL
+  const int32_t* W_h;   // [Hq] or NULL
+  const int32_t* k_h;   // [Hq] or NULL
+  float* mass;          // [B*Hq*nq, 4] or NULL
+  float* lse;           // [B*Hq*nq] or NULL
+  float2* cand_ml;      // [B*Hq*nq] log2-domain (max, sum) over the
+                        // candidates, when mass or lse is asked (workspace)
   void* O;
   int o_bf16;
   int32_t* idx;
@@ -29,11 +37,12 @@ struct PrefillArgs {
   uint64_t stall_ns;    // failure-path test hook (0: off)
 };
 
-// Bytes of the per-row Top-k key area at the start of the workspace body.
-size_t prefill_topk_bytes(int B, int n, int Hq, int k);
-// Workspace bytes beyond the status area.
-size_t prefill_workspace(bool bf16, int B, int n, int Hq, int Hkv, int d,
-                         int k);
+// Bytes of the per-row Top-k key area at the start of the workspace body
+// (rows = B*Hq*nq).
+size_t prefill_topk_bytes(int64_t rows, int k);
+// Workspace bytes beyond the status area: Top-k keys, the fallback row
+// list, the candidates' (max, sum) per row.
+size_t prefill_workspace(int64_t rows, int k);
 cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,
                            cudaStream_t stream);
 

@@ -34,7 +34,7 @@ def test_header_lists_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     for name in header_functions():
         assert hasattr(lib, name), name
-    assert lib.condensate_attn_version() == 100
+    assert lib.condensate_attn_version() == 200
 
 
 def test_status_strings(lib):

@@ -43,6 +43,8 @@ MUTATIONS = {
                                       "diag[DG_BOUND] = gam * amax_sel;"),
     "bound_ten_times_too_large": ("diag[DG_BOUND] = gam * (amax_sel + amax_unsel);",
                                   "diag[DG_BOUND] = 10.0 * gam * (amax_sel + amax_unsel);"),
+    "lse_max_dropped": ("if (diag) diag[DG_LSE] = mx + log(den);",
+                        "if (diag) diag[DG_LSE] = log(den);"),
     "score_term_dropped": ("for (int l = 0; l < d; ++l) acc += (double)q[l] * (double)kj[l];",
                            "for (int l = 1; l < d; ++l) acc += (double)q[l] * (double)kj[l];"),
 }

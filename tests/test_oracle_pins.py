@@ -211,7 +211,8 @@ def test_two_term_closed_form():
 def test_uniform_scores_closed_forms():
     """All keys equal: A is uniform, anchor mass 1/(i+1), window mass
     min(W, i+1)/(i+1), Top-k = [1..m_i] by the tie rule, sparse output = mean
-    of V over C_i, full output = mean of V over [0, i]."""
+    of V over C_i, full output = mean of V over [0, i], and the softmax
+    normaliser log sum_j exp(s_j) = s + log(i+1) with s = q.k/sqrt(d)."""
     n, d, W, k = 150, 8, 10, 7
     Q = _rand((1, 1, n, d), 14)
     K = np.tile(_rand((1, 1, 1, d), 15), (1, 1, n, 1))
@@ -229,6 +230,10 @@ def test_uniform_scores_closed_forms():
             min(W, i + 1) / (i + 1), rel=1e-12)
         assert out["excluded_mass"][i] == pytest.approx(
             (i + 1 - c) / (i + 1), abs=1e-12)
+        s_i = float(np.dot(Q[0, 0, i].astype(np.float64),
+                           K[0, 0, 0].astype(np.float64))) / math.sqrt(d)
+        assert out["lse"][i] == pytest.approx(s_i + math.log(i + 1),
+                                              rel=1e-12, abs=1e-12)
         np.testing.assert_allclose(out["o"][i],
                                    V[0, 0, s].astype(np.float64).mean(0),
                                    rtol=1e-12, atol=1e-13)

@@ -56,9 +56,9 @@ def test_decode_carried_scores(name):
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     ca.condensate_attn_decode(q, K, V, w.W, w.k, workspace=ws)
     assert ca.condensate_attn_status(ws) == ca.CA_OK
-    body = ws[256:].cpu().numpy().view(np.uint64)
-    per_head = body.size // (w.B * w.Hq)
-    assert per_head % w.k == 0 and per_head * w.B * w.Hq == body.size
+    nch = ca.condensate_attn_decode_chunks(w.B, w.n, w.Hkv, w.k)
+    per_head = nch * w.k
+    body = ws[256:256 + w.B * w.Hq * per_head * 8].cpu().numpy().view(np.uint64)
     G = w.Hq // w.Hkv
     total = 0
     for b in range(w.B):
