@@ -122,7 +122,6 @@ struct TcShared {
   int hi[kTileRows];
   float L[kTileRows];
   float M[kTileRows];       // row maximum over the candidates (mass reports)
-  float xsum[kSelThreads];  // per thread: sum of 2^((s - M) log2e/sqrt(d))
   short cnt[kSelThreads];   // entries in the thread's own segment, -1: overflow
   short xcnt[kSelThreads];  // entries in its spare segment
   signed char xcol[kSelThreads];  // spare segment index, -1: none
@@ -666,7 +665,11 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sh.cnt[col] = ovf ? (short)-1 : (short)(xc < 0 ? last : own);
     sh.xcnt[col] = (short)(xc < 0 ? 0 : last);
     sh.xcol[col] = (signed char)xc;
-    if constexpr (MASS) sh.xsum[col] = xs;
+    // per thread: sum of 2^((s - M) log2e/sqrt(d)) over its candidates, in
+    // the Q tile's bytes (every MMA reading them has completed: this
+    // thread consumed the last accumulator)
+    float* xsum = reinterpret_cast<float*>(sQ);
+    if constexpr (MASS) xsum[col] = xs;
     SelBar::sync();
     // ---- exact Top-k per row: four lanes per row, eight rows per warp
     {
@@ -685,7 +688,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         live = false;
       }
       if constexpr (MASS) {
-        float t = sh.xsum[part * kTileRows + row];
+        float t = reinterpret_cast<const float*>(sQ)[part * kTileRows + row];
         t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
         t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
         if (r < a.nq && part == 0)
@@ -1232,7 +1235,7 @@ constexpr int kMmaWarps = 4;  // 16 query rows each
 // keys as loaded in step 1.
 template <int D>
 struct MmaGatherSmem {
-  static constexpr size_t state = (size_t)16 * D * 4 + 2 * 16 * 4;
+  static constexpr size_t state = (size_t)16 * D * 4 + 3 * 16 * 4;
   __host__ __device__ static size_t per_warp(int k) {
     return state + (size_t)16 * k * 8;
   }
@@ -1262,7 +1265,8 @@ prefill_gather_mma(PrefillArgs a) {
   float* s_o = reinterpret_cast<float*>(g_smem + wid * MmaGatherSmem<D>::per_warp(k));
   float* s_m = s_o + 16 * D;
   float* s_l = s_m + 16;
-  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_l + 16);  // [16][k]
+  float* s_lx = s_l + 16;  // window sums of the unrounded weights (reports)
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_lx + 16);  // [16][k]
   const int bh = blockIdx.y;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int g = h / (a.Hq / a.Hkv);
@@ -1343,6 +1347,7 @@ prefill_gather_mma(PrefillArgs a) {
     qa[ks][3] = ld_b32(Qg + (size_t)cb * D + c + 8);
   }
   float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+  float lax = 0.f, lbx = 0.f;  // the same sums over the unrounded weights
   float o[NT][4];
 #pragma unroll
   for (int nd = 0; nd < NT; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
@@ -1377,6 +1382,10 @@ prefill_gather_mma(PrefillArgs a) {
     const float sb = nb == -INFINITY ? 1.f : exp2f(mb - nb);
     la *= sa;
     lb *= sb;
+    if constexpr (MASS) {
+      lax *= sa;
+      lbx *= sb;
+    }
 #pragma unroll
     for (int nd = 0; nd < NT; ++nd) {
       o[nd][0] *= sa;
@@ -1398,6 +1407,10 @@ prefill_gather_mma(PrefillArgs a) {
       // the sums use the rounded weights, as the MMA does
       la += __uint_as_float(p[h8][0]) + __uint_as_float(p[h8][1]);
       lb += __uint_as_float(p[h8][2]) + __uint_as_float(p[h8][3]);
+      if constexpr (MASS) {
+        lax += p0 + p1;
+        lbx += p2 + p3;
+      }
     }
     // p * V, keys of the k8 step ordered (2t, 2t+1) -> (t, t+4) so that the
     // score fragment is the A fragment as it stands
@@ -1419,11 +1432,19 @@ prefill_gather_mma(PrefillArgs a) {
   la += __shfl_xor_sync(0xFFFFFFFFu, la, 2);
   lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 1);
   lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 2);
+  if constexpr (MASS) {
+    lax += __shfl_xor_sync(0xFFFFFFFFu, lax, 1);
+    lax += __shfl_xor_sync(0xFFFFFFFFu, lax, 2);
+    lbx += __shfl_xor_sync(0xFFFFFFFFu, lbx, 1);
+    lbx += __shfl_xor_sync(0xFFFFFFFFu, lbx, 2);
+  }
   if (tq == 0) {
     s_m[gr] = ma;
     s_m[gr + 8] = mb;
     s_l[gr] = la;
     s_l[gr + 8] = lb;
+    s_lx[gr] = lax;
+    s_lx[gr + 8] = lbx;
   }
 #pragma unroll
   for (int nd = 0; nd < NT; ++nd) {
@@ -1452,8 +1473,10 @@ prefill_gather_mma(PrefillArgs a) {
     const int w = row_window(a.W_i, (int64_t)b * nq + rc, a.W_h, h, a.W, L,
                              a.status, false);
     const int lo = ic - w + 1 > 0 ? ic - w + 1 : 0;
-    const float m_win = s_m[r], l_win = s_l[r];  // the window alone
-    float mrun = s_m[r], den = s_l[r], ov[DL];
+    const float m_win = s_m[r], l_win = s_lx[r];  // the window alone
+    // den: sum over C_i with the window's rounded weights (normalises the
+    // output); denx: the same with unrounded weights (mass reports)
+    float mrun = s_m[r], den = s_l[r], denx = s_lx[r], ov[DL];
 #pragma unroll
     for (int e = 0; e < DL; ++e) ov[e] = s_o[r * D + sub * DL + e];
     float qv[DL];
@@ -1470,6 +1493,7 @@ prefill_gather_mma(PrefillArgs a) {
       const float mn = fmaxf(mrun, cm);
       const float f = exp2f(mrun - mn);
       den *= f;
+      if constexpr (MASS) denx *= f;
 #pragma unroll
       for (int e = 0; e < DL; ++e) ov[e] *= f;
 #pragma unroll
@@ -1478,6 +1502,7 @@ prefill_gather_mma(PrefillArgs a) {
         float vf[DL];
         vr[u].to_f32(vf);
         den += pw;
+        if constexpr (MASS) denx += pw;
 #pragma unroll
         for (int e = 0; e < DL; ++e) ov[e] = fmaf(pw, vf[e], ov[e]);
       }
@@ -1521,6 +1546,7 @@ prefill_gather_mma(PrefillArgs a) {
         float vf[DL];
         v0r.to_f32(vf);
         den = den * f + pw;
+        if constexpr (MASS) denx = denx * f + pw;
 #pragma unroll
         for (int e = 0; e < DL; ++e) ov[e] = fmaf(pw, vf[e], ov[e] * f);
         mrun = mn;
@@ -1531,8 +1557,8 @@ prefill_gather_mma(PrefillArgs a) {
           wa.merge(m_win, l_win);
           if (lo > 0) wa.add(d0 * sl2);
           const float2 cm = a.cand_ml[row];
-          mass_report(a.mass, a.lse, (size_t)row, mrun, den, wa.m, wa.l, cm.x,
-                      cm.y, d0 * sl2, lo > 0);
+          mass_report(a.mass, a.lse, (size_t)row, mrun, denx, wa.m, wa.l,
+                      cm.x, cm.y, d0 * sl2, lo > 0);
         }
       }
     }
