@@ -4,18 +4,8 @@
 // on the subset).
 //
 // Launch 1 (score + select), one CTA per 128-query tile of one (batch, head):
-//   bf16: warp-specialised tcgen05 pipeline.  Warp 0 issues TMA loads of the
-//         Q tile (once) and of 128-key K tiles into a ring of shared-memory
-//         stages, twice over (two passes); warp 1 issues tcgen05.mma (M=128,
-//         N=128, K=16 steps, bf16 in, fp32 out) into four TMEM accumulators;
-//         sixteen selector warps read the scores back with tcgen05.ld (thread
-//         = query row x 32-column chunk group).  Pass 1 keeps 128 column-slot
-//         maxima per row, whose k-th largest bounds the row's k-th best score
-//         from below; pass 2 appends every candidate at or above the bound to
-//         the thread's shared-memory segment; the exact Top-k is then cut per
-//         row.  Only key tiles that hold candidates of some row of the tile
-//         are computed, and the score matrix never leaves the SM.  Rows whose
-//         segments overflow go to an exact CUDA-core fallback.
+//   bf16: the tcgen05 pipeline of prefill_tc.cu; rows whose candidates
+//         overflowed its buffers go to the exact CUDA-core fallback here.
 //   fp32: a per-row heap selector fed by an FFMA dot-product loop over
 //         32-key tiles staged in shared memory (no TF32, so selection stays
 //         exact).
@@ -23,11 +13,10 @@
 //   C_i (ascending) and |C_i|, and run an fp32 online softmax over
 //   {0} U Top-k U window, re-using the selector's fp32 scores for Top-k.
 //   bf16 runs the window on warp-level MMA, 16 query rows per warp.
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "launch.cuh"
 #include "prefill.cuh"
+#include "prefill_rows.cuh"
 #include "profile.cuh"
 #include "row_topk.cuh"
 #include "select.cuh"
@@ -37,679 +26,6 @@
 namespace ca {
 
 namespace {
-
-// ------------------------------------------------------------ shared prologue
-// Window and last candidate position of each row of the tile (query rows
-// r0 .. r0+127 of head h, at positions p0 + r); returns the largest
-// last-candidate position over the tile's rows (-1 if none).
-__device__ void tile_rows(const PrefillArgs& a, int b, int h, int r0,
-                          int* s_hi, int* s_maxhi) {
-  const int tid = threadIdx.x;
-  if (tid == 0) *s_maxhi = -1;
-  __syncthreads();
-  if (tid < kTileRows) {
-    const int r = r0 + tid;
-    int hi = -1;
-    if (r < a.nq) {
-      const int w = row_window(a.W_i, (int64_t)b * a.nq + r, a.W_h, h, a.W,
-                               a.L, a.status, true);
-      hi = a.p0 + r - w;
-    }
-    s_hi[tid] = hi;
-    atomicMax(s_maxhi, hi);
-  }
-  __syncthreads();
-}
-
-// ============================================================ tcgen05 kernel
-// Two passes over the row tile's key tiles (the tensor pipe has room for
-// them; the selector is what costs):
-//   pass 1: every selector thread keeps, for its query row, the maximum over
-//           each of 32 column positions of its 32-column chunk of every key
-//           tile (128 slots per row over the four chunk groups).  The k-th
-//           largest slot maximum L is a lower bound of the row's k-th best
-//           score: the top k slots are k distinct candidates, all >= L.
-//   pass 2: recompute the scores and append every candidate with score >= L
-//           to the thread's own segment (about 1.1-1.4 k entries per row on
-//           random data), with predicated stores and no atomics.
-// The exact Top-k is then found per row by one warp (bisection on the key
-// bits over the row's four segments).  A row whose segment would overflow is
-// listed for an exact CUDA-core fallback.
-constexpr int kSelWarps = 16;                       // 4 chunk groups x 4 quarters
-constexpr int kSelThreads = 32 * kSelWarps;         // (row, chunk group) pairs
-constexpr int kTcThreads = 64 + kSelThreads;        // + TMA warp + MMA warp
-constexpr int kTmemBufs = 4;                        // 128-column accumulators
-constexpr int kMinSeg = 16;                         // smallest segment (entries)
-constexpr int kPoolCols = 16;                       // spare segments per CTA
-constexpr int kSegCols = kSelThreads + kPoolCols;   // segment columns
-constexpr int kScoreStride = (kSegCols + 1) * 4;    // bytes between positions
-constexpr int kCodeStride = (kSegCols + 2) * 2;     // (odd word strides: the
-                                                    //  entries of one column
-                                                    //  spread over the banks)
-constexpr uint32_t kMaskedScore = 0x7FC00000u;      // NaN: never >= L, ignored
-                                                    // by fmaxf
-using SelBar = GroupBarrier<1, kSelThreads>;
-
-template <int D>
-struct TcLayout {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int KB = D / 64;                   // 128-byte column blocks
-  static constexpr int NS = (D == 64) ? 4 : 2;        // K stages
-  static constexpr uint32_t kQBytes = BM * D * 2;
-  static constexpr uint32_t kKBytes = BN * D * 2;
-  static constexpr uint32_t kBlockBytes = 128 * 128;  // 128 rows x 128 bytes
-  static constexpr size_t q_off = 0;
-  static constexpr size_t k_off = q_off + kQBytes;
-  static constexpr size_t seg_off = k_off + (size_t)NS * kKBytes;
-  // Segments: P positions of scores (u32) then of codes (u16); the pass-1
-  // slot table (128 rows x 128 fp32) uses the same bytes first.
-  __host__ __device__ static size_t code_off(int P) {
-    return seg_off + ((size_t)P * kScoreStride + 15) / 16 * 16;
-  }
-  __host__ __device__ static size_t bytes(int P) {
-    size_t seg = code_off(P) - seg_off + (size_t)P * kCodeStride;
-    if (seg < (size_t)kTileRows * 128 * 4) seg = (size_t)kTileRows * 128 * 4;
-    return seg_off + seg + 1024;  // + the manual 1024-byte alignment
-  }
-};
-
-struct TcShared {
-  uint64_t kfull[4], kempty[4], qfull, tfull[kTmemBufs], tempty[kTmemBufs];
-  uint64_t never;  // failure-path test hook: a barrier nothing signals
-  uint32_t tmem;
-  int abort;
-  int maxhi;
-  int hi[kTileRows];
-  float L[kTileRows];
-  float M[kTileRows];       // row maximum over the candidates (mass reports)
-  short cnt[kSelThreads];   // entries in the thread's own segment, -1: overflow
-  short xcnt[kSelThreads];  // entries in its spare segment
-  signed char xcol[kSelThreads];  // spare segment index, -1: none
-  int pool;                 // spare segments handed out
-};
-
-// Append (score, code) at the segment cursor when score >= L; predicated
-// stores, so a warp never branches on the comparison.
-__device__ __forceinline__ void seg_append(uint32_t& as, uint32_t& ac,
-                                           uint32_t bits, float L,
-                                           uint32_t code) {
-  asm volatile(
-      "{ .reg .pred p; .reg .b16 c;\n\t"
-      "setp.ge.f32 p, %2, %3;\n\t"
-      "cvt.u16.u32 c, %5;\n\t"
-      "@p st.shared.b32 [%0], %4;\n\t"
-      "@p st.shared.b16 [%1], c;\n\t"
-      "@p add.u32 %0, %0, %6;\n\t"
-      "@p add.u32 %1, %1, %7; }"
-      : "+r"(as), "+r"(ac)
-      : "f"(__uint_as_float(bits)), "f"(L), "r"(bits), "r"(code),
-        "n"(kScoreStride), "n"(kCodeStride)
-      : "memory");
-}
-
-// Append the 32 scores of one key tile chunk.  Cursors are checked every 8
-// columns: a cursor past `*_max` (8 positions before the end) is clamped
-// and `full` is set, and the caller redoes the tile elsewhere.
-__device__ __forceinline__ void append_tile(const uint32_t (&raw)[32],
-                                            uint32_t& as, uint32_t& ac,
-                                            float L, uint32_t cbase,
-                                            uint32_t as_max, uint32_t ac_max,
-                                            bool& full) {
-#pragma unroll
-  for (int x = 0; x < 32; ++x) {
-    seg_append(as, ac, raw[x], L, cbase + x);
-    if ((x & 7) == 7) {
-      full |= as > as_max;
-      as = min(as, as_max);
-      ac = min(ac, ac_max);
-    }
-  }
-}
-
-// Segments of one row: slot g < 4 is chunk group g's own segment (column
-// g * 128 + row), slot 4 + g its spare one (column 512 + spare index, empty
-// when there is none).  Entry f lives in the last slot s with start[s] <= f
-// (empty slots share the start of the next one).
-struct RowSegs {
-  int n;           // entries of the row
-  int row;         // row within the tile
-  int start[8];    // prefix of the slot counts
-  int xcolm[4];    // spare segment column of each group
-  bool bad;        // a segment overflowed
-};
-
-__device__ __forceinline__ void row_segs(const TcShared& sh, int row,
-                                         RowSegs& q) {
-  q.row = row;
-  q.n = 0;
-  q.bad = false;
-#pragma unroll
-  for (int gq = 0; gq < 4; ++gq) {
-    const int c = sh.cnt[gq * kTileRows + row];
-    q.bad |= c < 0;
-    q.start[gq] = q.n;
-    q.n += c < 0 ? 0 : c;
-  }
-#pragma unroll
-  for (int gq = 0; gq < 4; ++gq) {
-    const int x = sh.xcol[gq * kTileRows + row];
-    q.start[4 + gq] = q.n;
-    q.xcolm[gq] = kSelThreads + (x < 0 ? 0 : x);
-    if (x >= 0) q.n += sh.xcnt[gq * kTileRows + row];
-  }
-}
-
-__device__ __forceinline__ void seg_locate(const RowSegs& rs, int f, int& col,
-                                           int& grp, int& e) {
-  int s = 0;
-#pragma unroll
-  for (int q = 1; q < 8; ++q) s += f >= rs.start[q];
-  int st = rs.start[0];
-#pragma unroll
-  for (int q = 1; q < 8; ++q)
-    if (q == s) st = rs.start[q];
-  int xcol = rs.xcolm[0];
-#pragma unroll
-  for (int q = 1; q < 4; ++q)
-    if (q == (s & 3)) xcol = rs.xcolm[q];
-  grp = s & 3;
-  col = s < 4 ? grp * kTileRows + rs.row : xcol;
-  e = f - st;
-}
-
-__device__ __forceinline__ uint32_t seg_hi(const unsigned char* seg, int col,
-                                           int e) {
-  const uint32_t bits = *reinterpret_cast<const uint32_t*>(
-      seg + (size_t)e * kScoreStride + col * 4);
-  return ord_f32(__uint_as_float(bits));
-}
-
-__device__ __forceinline__ uint32_t seg_lo(const unsigned char* codes,
-                                           int col, int grp, int e) {
-  const uint32_t code = *reinterpret_cast<const uint16_t*>(
-      codes + (size_t)e * kCodeStride + col * 2);
-  const uint32_t j = (code >> 5) * 128 + grp * 32 + (code & 31);
-  return 0xFFFFFFFFu - j;
-}
-
-// Sum over the four lanes of a row group.
-__device__ __forceinline__ int quad_sum(int v) {
-  v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-  return v + __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-}
-
-// Exact Top-k of the rows of one warp, four lanes per row (lane & 3 = part;
-// entry f of the row is held by part f & 3).  `sel` rows take the k largest
-// keys (ord(score), ~j) of their n entries, found by bisection on the score
-// bits (and on the index bits only when equal scores straddle the cut);
-// `all` rows (n <= k) take every entry.  The selected keys go to out[0..) in
-// any order, padded with empty keys.  Missing entries hold 0, below every
-// probe.
-template <int NE>
-__device__ __forceinline__ void quad_select(const unsigned char* seg,
-                                            const unsigned char* codes,
-                                            const RowSegs& rs, bool live,
-                                            uint32_t lob, int k, int kpad,
-                                            uint64_t* out, int part) {
-  uint32_t hv[NE];
-#pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    const int f = part + 4 * t;
-    hv[t] = 0u;
-    if (live && f < rs.n) {
-      int col, grp, e;
-      seg_locate(rs, f, col, grp, e);
-      hv[t] = seg_hi(seg, col, e);
-    }
-  }
-  const bool sel = live && rs.n > k;
-  // bisection start: the common high bits of the bound and the row maximum
-  uint32_t mx = 0u;
-#pragma unroll
-  for (int t = 0; t < NE; ++t) mx = max(mx, hv[t]);
-  mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-  mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-  const uint32_t diff = lob ^ mx;
-  const int nb = sel ? (diff ? 32 - __clz(diff) : 0) : 0;
-  uint32_t tau = nb == 32 ? 0u : (lob >> nb) << nb;
-  bool done = nb == 0, exact = false;
-  const int bmax = __reduce_max_sync(0xFFFFFFFFu, nb);
-#pragma unroll 1
-  for (int b = bmax - 1; b >= 0; --b) {
-    if (__all_sync(0xFFFFFFFFu, done)) break;
-    const uint32_t c = tau | (1u << b);
-    int m = 0;
-#pragma unroll
-    for (int t = 0; t < NE; ++t) m += hv[t] >= c;
-    m = quad_sum(m);
-    const bool up = !done && b < nb && m >= k;
-    tau = up ? c : tau;
-    const bool fin = up && m == k;
-    done |= fin;
-    exact |= fin;
-  }
-  uint32_t th_hi = sel ? tau : 0u, th_lo = 0u;
-  // equal scores straddling the cut: the lower positions win
-  int gt = 0, ge = 0;
-#pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    gt += hv[t] > th_hi;
-    ge += hv[t] >= th_hi;
-  }
-  gt = quad_sum(gt);
-  ge = quad_sum(ge);
-  const int need = (sel && !exact && ge > k) ? k - gt : 0;
-  if (__any_sync(0xFFFFFFFFu, need > 0)) {
-    uint32_t lo[NE];
-#pragma unroll
-    for (int t = 0; t < NE; ++t) {
-      const int f = part + 4 * t;
-      lo[t] = 0u;
-      if (need > 0 && f < rs.n && hv[t] == th_hi) {
-        int col, grp, e;
-        seg_locate(rs, f, col, grp, e);
-        lo[t] = seg_lo(codes, col, grp, e);
-      }
-    }
-#pragma unroll 1
-    for (int b = 31; b >= 0; --b) {
-      const uint32_t c = th_lo | (1u << b);
-      int m = 0;
-#pragma unroll
-      for (int t = 0; t < NE; ++t) m += hv[t] == th_hi && lo[t] >= c;
-      m = quad_sum(m);
-      th_lo = (need > 0 && m >= need) ? c : th_lo;
-    }
-  }
-  // write the selected keys: exclusive prefix over the four parts
-  int cnt = 0;
-#pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    const int f = part + 4 * t;
-    if (live && f < rs.n && hv[t] >= th_hi) {
-      bool s = hv[t] > th_hi || th_lo == 0u;
-      if (!s) {
-        int col, grp, e;
-        seg_locate(rs, f, col, grp, e);
-        s = seg_lo(codes, col, grp, e) >= th_lo;
-      }
-      cnt += s;
-    }
-  }
-  const int up1 = __shfl_up_sync(0xFFFFFFFFu, cnt, 1);
-  const int up2 = __shfl_up_sync(0xFFFFFFFFu, cnt, 2);
-  const int up3 = __shfl_up_sync(0xFFFFFFFFu, cnt, 3);
-  const int pre =
-      (part >= 1 ? up1 : 0) + (part >= 2 ? up2 : 0) + (part >= 3 ? up3 : 0);
-  const int total = quad_sum(cnt);
-  if (live) {
-    int pos = pre;
-#pragma unroll
-    for (int t = 0; t < NE; ++t) {
-      const int f = part + 4 * t;
-      if (f < rs.n && hv[t] >= th_hi) {
-        int col, grp, e;
-        seg_locate(rs, f, col, grp, e);
-        const uint32_t lo = seg_lo(codes, col, grp, e);
-        if (hv[t] > th_hi || lo >= th_lo) {
-          out[pos++] = ((uint64_t)hv[t] << 32) | lo;
-        }
-      }
-    }
-    for (int e = total + part; e < kpad; e += 4) out[e] = 0ull;
-  }
-}
-
-template <int D, bool MASS>
-__global__ void __launch_bounds__(kTcThreads, 1)
-prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
-                      int P) {
-  using Lay = TcLayout<D>;
-  constexpr int BN = Lay::BN, NS = Lay::NS, KB = Lay::KB;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = smem + Lay::q_off;
-  unsigned char* sK = smem + Lay::k_off;
-  unsigned char* seg = smem + Lay::seg_off;     // scores [P][512] (stride 513)
-  unsigned char* codes = smem + Lay::code_off(P);  // codes [P][512] (514)
-  float* table = reinterpret_cast<float*>(seg);  // pass-1 slots, then free
-  __shared__ TcShared sh;
-
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (a.Hq / a.Hkv);
-  const int i0 = qt * Lay::BM;  // first query row of the tile
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int k = head_k(a.k_h, h, a.k, a.status, qt == 0 && tid == 0);
-
-  tile_rows(a, b, h, i0, sh.hi, &sh.maxhi);
-  if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      sm100::mbar_init(&sh.kfull[s], 1);
-      sm100::mbar_init(&sh.kempty[s], 1);
-    }
-    sm100::mbar_init(&sh.qfull, 1);
-    sm100::mbar_init(&sh.never, 1);
-    for (int t = 0; t < kTmemBufs; ++t) {
-      sm100::mbar_init(&sh.tfull[t], 1);
-      sm100::mbar_init(&sh.tempty[t], kSelWarps);
-    }
-    sh.abort = 0;
-    sh.pool = 0;
-    sm100::fence_barrier_init();
-  }
-  if (warp == 1) {
-    sm100::tmem_alloc(&sh.tmem, kTmemBufs * BN);
-    sm100::tmem_relinquish();
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tmem = sh.tmem;
-  const int maxhi = sh.maxhi;
-  const int T = maxhi >= 1 ? maxhi / BN + 1 : 0;  // key tiles with candidates
-  const int TT = 2 * T;                           // two passes
-  volatile int* abort_flag = &sh.abort;
-
-  if (warp == 0) {
-    // ---------------- TMA producer: key tiles 0..T-1, twice
-    if (lane == 0 && T > 0) {
-      sm100::prefetch_tmap(&tmQ);
-      sm100::prefetch_tmap(&tmK);
-      const int qrow = ((b * a.Hq + h) * a.nq) + i0;
-      const int krow = (b * a.Hkv + g) * a.L;
-      sm100::mbar_arrive_expect_tx(&sh.qfull, Lay::kQBytes);
-      for (int kb = 0; kb < KB; ++kb)
-        sm100::tma_load_2d(sQ + kb * Lay::kBlockBytes, &tmQ, &sh.qfull, kb * 64,
-                           qrow);
-      int issued = 0;
-      int s = 0;
-      uint32_t ph = 0;
-      for (int t = 0; t < TT; ++t) {
-        const int tile = t < T ? t : t - T;
-        if (t >= NS &&
-            !sm100::wait_or_abort(&sh.kempty[s], ph ^ 1, abort_flag, a.status,
-                                   a.wait_ns))
-          break;
-        sm100::mbar_arrive_expect_tx(&sh.kfull[s], Lay::kKBytes);
-        unsigned char* dst = sK + (size_t)s * Lay::kKBytes;
-        for (int kb = 0; kb < KB; ++kb)
-          sm100::tma_load_2d(dst + kb * Lay::kBlockBytes, &tmK, &sh.kfull[s],
-                             kb * 64, krow + tile * BN);
-        issued = t + 1;
-        if (++s == NS) {
-          s = 0;
-          ph ^= 1;
-        }
-      }
-      // Let every copy this thread started land before the CTA can exit.
-      bool drained = sm100::mbar_wait(&sh.qfull, 0, kDrainWaitNs);
-      for (int t = issued - NS < 0 ? 0 : issued - NS; t < issued; ++t)
-        drained &= sm100::mbar_wait(&sh.kfull[t % NS], (t / NS) & 1,
-                                    kDrainWaitNs);
-      if (!drained) raise_flag(a.status, kErrTimeout);
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0 && T > 0) {
-      constexpr uint32_t idesc = sm100::idesc_bf16_f32(Lay::BM, BN);
-      const uint32_t aq = sm100::smem_u32(sQ);
-      const uint32_t ak = sm100::smem_u32(sK);
-      int done = 0;
-      if (a.stall_ns) {
-        // Failure-path test hook: wait on a barrier that nothing signals, so
-        // the wait runs out, raises the time-out flag and aborts every wait
-        // of the CTA; the kernel then leaves through its normal path.
-        sm100::wait_or_abort(&sh.never, 0, abort_flag, a.status, a.stall_ns);
-      }
-      if (sm100::wait_or_abort(&sh.qfull, 0, abort_flag, a.status, a.wait_ns)) {
-        int s = 0;
-        uint32_t ph = 0;
-        for (int t = 0; t < TT; ++t) {
-          const int buf = t & (kTmemBufs - 1);
-          if (!sm100::wait_or_abort(&sh.kfull[s], ph, abort_flag, a.status,
-                                    a.wait_ns))
-            break;
-          if (t >= kTmemBufs &&
-              !sm100::wait_or_abort(&sh.tempty[buf], ((t / kTmemBufs) & 1) ^ 1,
-                                    abort_flag, a.status, a.wait_ns))
-            break;
-          sm100::tc_fence_after();
-          const uint32_t d_tmem = tmem + buf * BN;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Lay::kBlockBytes + (kk & 3) * 32;
-            sm100::mma_bf16(d_tmem, sm100::desc_k_sw128(aq + off),
-                            sm100::desc_k_sw128(ak + s * Lay::kKBytes + off),
-                            idesc, kk > 0 ? 1u : 0u);
-          }
-          sm100::mma_commit(&sh.kempty[s]);
-          sm100::mma_commit(&sh.tfull[buf]);
-          done = t + 1;
-          if (++s == NS) {
-            s = 0;
-            ph ^= 1;
-          }
-        }
-      }
-      // The last commit covers every MMA issued: wait for it before exit.
-      if (done > 0 &&
-          !sm100::mbar_wait(&sh.tfull[(done - 1) & (kTmemBufs - 1)],
-                            ((done - 1) / kTmemBufs) & 1, kDrainWaitNs))
-        raise_flag(a.status, kErrTimeout);
-    }
-  } else {
-    // ---------------- selector warps: thread = (query row, chunk group)
-    const int sw = warp - 2;               // 0..15
-    const int grp = sw >> 2;               // 32-column chunk of every tile
-    const int quarter = warp & 3;          // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;
-    const int col = grp * kTileRows + r;   // this thread's segment column
-    const int hi = sh.hi[r];
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + grp * 32;
-
-    // Scores of key tile t for this thread's row and chunk, with
-    // non-candidates (j = 0, the window, the future) replaced by NaN.
-    auto fetch = [&](int t, uint32_t (&raw)[32]) -> bool {
-      const int buf = t & (kTmemBufs - 1);
-      if (!__all_sync(0xFFFFFFFFu,
-                      sm100::wait_or_abort(&sh.tfull[buf], (t / kTmemBufs) & 1,
-                                           abort_flag, a.status, a.wait_ns)))
-        return false;
-      sm100::tc_fence_after();
-      sm100::tmem_ld_32x32b_x32(tl + buf * BN, raw);
-      sm100::tmem_wait_ld();
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&sh.tempty[buf]);
-      return true;
-    };
-
-    // ---- pass 1: slot maxima
-    float colmax[32];
-#pragma unroll
-    for (int x = 0; x < 32; ++x) colmax[x] = -INFINITY;
-    int t = 0;
-    for (; t < T; ++t) {
-      uint32_t raw[32];
-      if (!fetch(t, raw)) break;
-      const int j0 = t * BN + grp * 32;
-      if (!(j0 >= 1 && j0 + 31 <= hi)) {
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (!(j0 + x >= 1 && j0 + x <= hi)) raw[x] = kMaskedScore;
-      }
-#pragma unroll
-      for (int x = 0; x < 32; ++x)
-        colmax[x] = fmaxf(colmax[x], __uint_as_float(raw[x]));
-    }
-    // ---- bound: k-th largest of the row's 128 slot maxima.  The table
-    // row is stored with its 16-byte pieces XOR-swizzled by the row index so
-    // that 32 rows written (or one row read) at once spread over the banks.
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int piece = (grp * 8 + c) ^ (r & 31);
-      *reinterpret_cast<float4*>(table + r * 128 + piece * 4) =
-          make_float4(colmax[4 * c], colmax[4 * c + 1], colmax[4 * c + 2],
-                      colmax[4 * c + 3]);
-    }
-    SelBar::sync();
-    {
-      // Four lanes per row (part = slots part*32 .. part*32+31), eight rows
-      // per warp.  tau is the largest value with its low 14 bits zero and at
-      // least k slots >= tau (or the first probe that leaves exactly k); any
-      // such tau is a valid bound.
-      const int row = sw * 8 + (lane >> 2), part = lane & 3;
-      uint32_t key[32];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int piece = (part * 8 + c) ^ (row & 31);
-        const float4 v = *reinterpret_cast<const float4*>(table + row * 128 +
-                                                           piece * 4);
-        key[4 * c] = ord_f32(v.x);
-        key[4 * c + 1] = ord_f32(v.y);
-        key[4 * c + 2] = ord_f32(v.z);
-        key[4 * c + 3] = ord_f32(v.w);
-      }
-      uint32_t tau = 0u;
-      bool done = false;
-#pragma unroll 1
-      for (int bit = 31; bit >= 14; --bit) {
-        const uint32_t c = tau | (1u << bit);
-        int m = 0;
-#pragma unroll
-        for (int x = 0; x < 32; ++x) m += key[x] >= c;
-        m = quad_sum(m);
-        const bool up = !done && m >= k;
-        tau = up ? c : tau;
-        done |= up && m == k;
-        if (__all_sync(0xFFFFFFFFu, done)) break;
-      }
-      if (part == 0)
-        sh.L[row] = k == 0 ? INFINITY  // nothing to select: no appends
-                    : (tau <= ord_f32(-INFINITY)) ? -INFINITY
-                                                  : unord_f32(tau);
-      if constexpr (MASS) {
-        uint32_t mx = 0u;
-#pragma unroll
-        for (int x = 0; x < 32; ++x) mx = max(mx, key[x]);
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-        if (part == 0) sh.M[row] = unord_f32(mx);
-      }
-    }
-    SelBar::sync();
-    const float Lr = sh.L[r];
-    const float sl2 = 1.4426950408889634f / sqrtf((float)D);
-    const float Mr = MASS ? sh.M[r] : 0.f;
-    float xs = 0.f;  // this thread's share of the candidates' sum
-    // ---- pass 2: append every candidate >= L to this thread's segment; a
-    // full segment continues in a spare one (rare), else the row is listed
-    // for the exact fallback.
-    const uint32_t seg_s = sm100::smem_u32(seg), seg_c = sm100::smem_u32(codes);
-    uint32_t as0 = seg_s + col * 4, ac0 = seg_c + col * 2;
-    // cursors are checked every 8 columns so that 8 more entries still fit
-    uint32_t as_max = as0 + (uint32_t)(P - 8) * kScoreStride;
-    uint32_t ac_max = ac0 + (uint32_t)(P - 8) * kCodeStride;
-    uint32_t as = as0, ac = ac0;
-    int xc = -1, own = 0;
-    bool ovf = false;
-    for (; t < TT; ++t) {
-      uint32_t raw[32];
-      if (!fetch(t, raw)) break;
-      const int tile = t - T;
-      const int j0 = tile * BN + grp * 32;
-      if (!(j0 >= 1 && j0 + 31 <= hi)) {
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (!(j0 + x >= 1 && j0 + x <= hi)) raw[x] = kMaskedScore;
-      }
-      if constexpr (MASS) {
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          xs += exp2f(fmaxf((__uint_as_float(raw[x]) - Mr) * sl2, -INFINITY));
-      }
-      const uint32_t cbase = (uint32_t)tile * 32;
-      const uint32_t as_t = as;  // cursor at the tile start
-      bool full = false;
-      append_tile(raw, as, ac, Lr, cbase, as_max, ac_max, full);
-      if (__any_sync(0xFFFFFFFFu, full)) {
-        // An own segment is full: drop this tile's entries from it and redo
-        // the tile in a spare segment (once per thread, while any is left);
-        // otherwise the row goes to the exact fallback.  The whole warp runs
-        // the redo; threads with nothing to redo append nothing (L = +inf).
-        float Lredo = INFINITY;
-        if (full) {
-          const int px = (xc < 0 && !ovf) ? atomicAdd(&sh.pool, 1) : kPoolCols;
-          if (px < kPoolCols) {
-            own = (as_t - as0) / kScoreStride;
-            xc = px;
-            as0 = seg_s + (kSelThreads + px) * 4;
-            ac0 = seg_c + (kSelThreads + px) * 2;
-            as_max = as0 + (uint32_t)(P - 8) * kScoreStride;
-            ac_max = ac0 + (uint32_t)(P - 8) * kCodeStride;
-            as = as0;
-            ac = ac0;
-            Lredo = Lr;
-          } else {
-            ovf = true;
-          }
-        }
-        bool full2 = false;
-        append_tile(raw, as, ac, Lredo, cbase, as_max, ac_max, full2);
-        ovf |= full2;
-      }
-    }
-    const int last = (as - as0) / kScoreStride;
-    sh.cnt[col] = ovf ? (short)-1 : (short)(xc < 0 ? last : own);
-    sh.xcnt[col] = (short)(xc < 0 ? 0 : last);
-    sh.xcol[col] = (signed char)xc;
-    // per thread: sum of 2^((s - M) log2e/sqrt(d)) over its candidates, in
-    // the Q tile's bytes (every MMA reading them has completed: this
-    // thread consumed the last accumulator)
-    float* xsum = reinterpret_cast<float*>(sQ);
-    if constexpr (MASS) xsum[col] = xs;
-    SelBar::sync();
-    // ---- exact Top-k per row: four lanes per row, eight rows per warp
-    {
-      const int row = sw * 8 + (lane >> 2), part = lane & 3;
-      const int r = i0 + row;
-      RowSegs rs;
-      row_segs(sh, row, rs);
-      const size_t grow = (size_t)(b * a.Hq + h) * a.nq + r;
-      bool live = r < a.nq;
-      if (live && (rs.bad || rs.n > 128)) {
-        // listed for the exact fallback pass; it writes this row
-        if (part == 0) {
-          const uint32_t pos = atomicAdd(a.ovf_count, 1u);
-          a.ovf_rows[pos] = (uint32_t)grow;
-        }
-        live = false;
-      }
-      if constexpr (MASS) {
-        float t = reinterpret_cast<const float*>(sQ)[part * kTileRows + row];
-        t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
-        t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
-        if (r < a.nq && part == 0)
-          a.cand_ml[grow] = make_float2(sh.M[row] * sl2, t);
-      }
-      const uint32_t lob = ord_f32(sh.L[row]);
-      uint64_t* out = a.topk + grow * a.k;
-      if (__all_sync(0xFFFFFFFFu, !live || rs.n <= 64))
-        quad_select<16>(seg, codes, rs, live, lob, k, a.k, out, part);
-      else
-        quad_select<32>(seg, codes, rs, live, lob, k, a.k, out, part);
-    }
-  }
-  __syncwarp();  // reconverge single-lane roles before the CTA barrier
-  sm100::tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, kTmemBufs * BN);
-  }
-}
 
 // Raw (undecoded) copy of DL consecutive elements of a row.
 template <typename T, int DL>
@@ -1572,69 +888,12 @@ prefill_gather_mma(PrefillArgs a) {
 }
 
 // ============================================================ host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
-                                &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// Row-major [rows, d] bf16 tensor, boxes of 128 rows x 64 columns, 128-byte
-// swizzle (matches the UMMA K-major SW128 descriptor).
-bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int d) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                   const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 bool want_mass(const PrefillArgs& a) {
   return a.mass != nullptr || a.lse != nullptr;
 }
 
 template <int D>
-cudaError_t launch_select_tc(const PrefillArgs& a, cudaStream_t s) {
-  using Lay = TcLayout<D>;
-  // segment codes hold tile * 32 + column in 16 bits
-  if ((a.L + Lay::BN - 1) / Lay::BN > 2048) return cudaErrorNotSupported;
-  CUtensorMap tq, tk;
-  if (!make_tmap(&tq, a.Q, (uint64_t)a.B * a.Hq * a.nq, D)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tk, a.K, (uint64_t)a.B * a.Hkv * a.L, D)) return cudaErrorInvalidValue;
-  // Segment positions per (row, chunk group) thread: about k/4 entries are
-  // expected (1.1-1.4 k per row), but one key tile can put 31 entries into
-  // one segment (rows with fewer than k candidates); the cursor check every
-  // 8 columns keeps 8 positions in reserve.
-  const size_t budget = 227 * 1024 - sizeof(TcShared);
-  int P = a.k > 32 ? 46 : 40;
-  while (P > kMinSeg && Lay::bytes(P) > budget) --P;
-  if (Lay::bytes(P) > budget || P < 40) return cudaErrorNotSupported;
-  const size_t smem = Lay::bytes(P);
-  auto kern = want_mass(a) ? prefill_score_topk_tc<D, true>
-                           : prefill_score_topk_tc<D, false>;
-  cudaError_t e = ensure_smem(kern, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((a.nq + 127) / 128, a.Hq, a.B);
-  prof_before(s, "prefill_score_topk_tc");
-  kern<<<grid, kTcThreads, smem, s>>>(tq, tk, a, P);
-  prof_after(s);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (a.k == 0) return cudaSuccess;  // run for the mass reports only
-  // rows whose segments overflowed (rare on typical inputs): exact fallback
+cudaError_t launch_overflow_d(const PrefillArgs& a, cudaStream_t s) {
   const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
   prof_before(s, "prefill_overflow_rows");
   prefill_overflow_rows<__nv_bfloat16, D><<<sm_count(), kFbThreads, fb_smem, s>>>(a);
@@ -1725,8 +984,15 @@ cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,
                            cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   if (a.k > 0 || want_mass(a)) {
-    if (bf16) e = d == 64 ? launch_select_tc<64>(a, s) : launch_select_tc<128>(a, s);
-    else e = d == 64 ? launch_select_f32<64>(a, s) : launch_select_f32<128>(a, s);
+    if (bf16) {
+      e = launch_select_tc(a, d, s);
+      // rows whose candidates overflowed their buffers (rare on typical
+      // inputs): the exact fallback
+      if (e == cudaSuccess && a.k > 0)
+        e = d == 64 ? launch_overflow_d<64>(a, s) : launch_overflow_d<128>(a, s);
+    } else {
+      e = d == 64 ? launch_select_f32<64>(a, s) : launch_select_f32<128>(a, s);
+    }
     if (e != cudaSuccess) return e;
   }
   if (bf16) e = d == 64 ? launch_gather_mma<64>(a, s) : launch_gather_mma<128>(a, s);

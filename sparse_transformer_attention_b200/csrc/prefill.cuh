@@ -45,5 +45,7 @@ size_t prefill_topk_bytes(int64_t rows, int k);
 size_t prefill_workspace(int64_t rows, int k);
 cudaError_t prefill_launch(const PrefillArgs& a, bool bf16, int d,
                            cudaStream_t stream);
+// The tensor-core score + Top-k pass (bf16 inputs; prefill_tc.cu).
+cudaError_t launch_select_tc(const PrefillArgs& a, int d, cudaStream_t stream);
 
 }  // namespace ca

@@ -108,6 +108,31 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
+// 3-D tiled load of one box into shared memory, completing on `bar`.
+// c0 is the innermost (element) coordinate, always 0 here.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m,
+                                            uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(m), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Two fp32 values rounded toward zero to bf16 and packed (hi, lo).
+__device__ __forceinline__ uint32_t cvt_rz_bf16x2(float hi, float lo) {
+  uint32_t r;
+  asm("cvt.rz.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Lane-wise maximum of two packed bf16 pairs (a NaN lane takes the other).
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Bulk (non-tensor) copy of `bytes` contiguous bytes from global to shared
 // memory, completing on `bar`.  Both addresses 16-byte aligned, bytes a
 // multiple of 16.  No multicast.
