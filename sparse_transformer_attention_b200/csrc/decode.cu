@@ -109,79 +109,6 @@ struct TopkShared {
                           // candidates' log2-scaled scores (mass reports)
 };
 
-// One warp cuts the list lst[0..n) of unique keys down to its best kk keys
-// (n > kk >= 1), in place and in no particular order, and returns the
-// threshold T with exactly kk keys >= T.  Radix select from the most
-// significant byte, stopping as soon as the chosen byte's bucket holds
-// exactly the keys still needed (its lower bound then separates the sets).
-__device__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint32_t* hist,
-                             int lane) {
-  uint64_t prefix = 0ull;
-  uint32_t need = (uint32_t)kk;
-#pragma unroll 1
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    const uint64_t hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
-#pragma unroll
-    for (int b = lane; b < 256; b += 32) hist[b] = 0u;
-    __syncwarp();
-    for (int e = lane; e < n; e += 32) {
-      const uint64_t key = lst[e];
-      if ((key & hmask) == prefix)
-        atomicAdd(&hist[(uint32_t)(key >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    uint32_t c[8], sum = 0;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      c[t] = hist[255 - 8 * lane - t];
-      sum += c[t];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    const uint32_t excl = incl - sum;
-    const bool mine = excl < need && need <= incl;
-    uint32_t digit = 0, nd = 0, bucket = 0;
-    if (mine) {
-      uint32_t acc = excl;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (acc + c[t] >= need) {
-          digit = 255u - 8u * lane - t;
-          nd = need - acc;
-          bucket = c[t];
-          break;
-        }
-        acc += c[t];
-      }
-    }
-    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
-    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
-    nd = __shfl_sync(0xFFFFFFFFu, nd, src);
-    bucket = __shfl_sync(0xFFFFFFFFu, bucket, src);
-    prefix |= (uint64_t)digit << shift;
-    need = nd;
-    __syncwarp();  // the histogram is cleared again next pass
-    if (bucket == nd) break;
-  }
-  // keep the keys >= prefix, packed to the front in reading order; a slot
-  // is only written after the whole group of 32 that covers it was read
-  int wr = 0;
-  for (int base = 0; base < n; base += 32) {
-    const int e = base + lane;
-    const uint64_t key = e < n ? lst[e] : 0ull;
-    const bool keep = e < n && key >= prefix;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-    if (keep) lst[wr + __popc(bal & ((1u << lane) - 1u))] = key;
-    wr += __popc(bal);
-    __syncwarp();
-  }
-  return prefix;
-}
-
 // At a check point (all inserts of the stretch done): warp h cuts list h
 // down to its head's k keys when it holds more than the limit: that k after
 // the first stretch (so that a useful threshold exists early), else the
@@ -760,17 +687,28 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   // with k = 0 the set is anchor and window only: the score pass runs only
   // for the mass reports (the candidates' sums)
   if (a.k > 0 || mass) {
-    auto k1 = mass ? decode_score_topk<T, D, G, true>
-                   : decode_score_topk<T, D, G, false>;
-    // the largest shared-memory carve-out, so that two CTAs fit per SM
-    e = ensure_smem(k1, smem1, true);
-    if (e != cudaSuccess) return e;
-    dim3 grid1(a.nchunks, a.Hkv, a.B);
-    prof_before(stream, "decode_score_topk");
-    k1<<<grid1, kThreads, smem1, stream>>>(a);
-    prof_after(stream);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    bool done = false;
+    if constexpr (sizeof(T) == 2) {
+      // bf16: the dot products on the tensor pipe
+      e = decode_score_tc_launch(a, D, mass, stream);
+      if (e != cudaErrorNotSupported) {
+        if (e != cudaSuccess) return e;
+        done = true;
+      }
+    }
+    if (!done) {
+      auto k1 = mass ? decode_score_topk<T, D, G, true>
+                     : decode_score_topk<T, D, G, false>;
+      // the largest shared-memory carve-out, so that two CTAs fit per SM
+      e = ensure_smem(k1, smem1, true);
+      if (e != cudaSuccess) return e;
+      dim3 grid1(a.nchunks, a.Hkv, a.B);
+      prof_before(stream, "decode_score_topk");
+      k1<<<grid1, kThreads, smem1, stream>>>(a);
+      prof_after(stream);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
   }
   const size_t smem2 = (size_t)a.nchunks * a.k * 8 + (size_t)a.kpow2 * 8 +
                        sizeof(SelectState<1>);
@@ -826,8 +764,9 @@ int decode_chunks(int B, int L, int Hkv, int k) {
 }
 
 int decode_chunk_len(int L, int nchunks) {
+  // a whole number of 128-key tiles of the tensor-core score pass
   int len = (L + nchunks - 1) / nchunks;
-  return (len + 63) / 64 * 64;
+  return (len + 127) / 128 * 128;
 }
 
 cudaError_t decode_launch(const DecodeArgs& a, bool bf16, int d,

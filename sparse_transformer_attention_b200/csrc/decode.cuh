@@ -43,6 +43,10 @@ struct DecodeArgs {
 };
 
 int decode_chunks(int B, int L, int Hkv, int k);
+// The bf16 score pass on tensor cores (decode_tc.cu); cudaErrorNotSupported
+// when its shared-memory plan does not fit (the CUDA-core pass runs then).
+cudaError_t decode_score_tc_launch(const DecodeArgs& a, int d, bool mass,
+                                   cudaStream_t stream);
 int decode_chunk_len(int L, int nchunks);
 cudaError_t decode_launch(const DecodeArgs& a, bool bf16, int d,
                           cudaStream_t stream);

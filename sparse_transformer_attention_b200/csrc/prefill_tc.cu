@@ -4,7 +4,7 @@
 // (identify the set, then attend on it).
 //
 // One CTA per 128-query tile of one (batch, head):
-//   TMA warps  the Q tile once, then the key tiles 0..T-1 twice (two passes)
+//   TMA warps  the key tiles 0..T-1 twice (two passes)
 //              through a ring of 32 KB stages, one stage per producer warp
 //              (three at d = 64, two at d = 128: warps 0, 2 and 3).  Every
 //              copy moves 32 KB (two 128-key tiles at d = 64, one tile with
@@ -15,7 +15,10 @@
 //              copies from two threads do).  At d = 64 a copy outlasts the MMAs
 //              of its two tiles, hence the third stage.
 //   warp 1     MMA: tcgen05.mma kind::f16, M = N = 128, bf16 in, fp32 out, into
-//              four 128-column TMEM accumulators.
+//              three 128-column TMEM accumulators.  A (the Q tile) is read
+//              from TMEM, where the first selector warps store it once (their
+//              rows, straight from global memory): that leaves its 16-32 KB of
+//              shared memory to the candidate segments.
 //   16 warps   selectors (after the TMA and MMA warps), thread = (query row,
 //              32-column chunk group of every
 //              key tile), reading the accumulators with tcgen05.ld 32x32b:
@@ -45,6 +48,7 @@
 #include "profile.cuh"
 #include "select.cuh"
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace ca {
 
@@ -54,7 +58,8 @@ constexpr int kBM = kPrefillTileRows;  // query rows per CTA
 constexpr int kBN = 128;               // keys per accumulator tile
 constexpr int kSelWarps = 16;          // 4 chunk groups x 4 TMEM lane quarters
 constexpr int kSelThreads = 32 * kSelWarps;
-constexpr int kTmemBufs = 4;
+constexpr int kTmemBufs = 3;
+constexpr int kQCol = kTmemBufs * 128;  // TMEM columns of the Q tile
 constexpr uint32_t kStageBytes = 32768;
 constexpr uint32_t kBlockBytes = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kPool = 16;                    // spare segments per CTA
@@ -63,7 +68,7 @@ constexpr int kSegCols = kSelThreads + kPool;
 // one position are contiguous (a warp's 32 threads at equal cursors store
 // 256 contiguous bytes), and positions are 2 banks apart.
 constexpr int kEntStride = (kSegCols + 1) * 8;
-constexpr int kCheck = 16;                   // columns between room checks
+constexpr int kCheck = 8;                    // columns between room checks
 constexpr int kCutNE = 40;                   // entries per lane in the cut
 constexpr uint32_t kMaskedScore = 0x7FC00000u;  // NaN: never >= L
 using SelBar = GroupBarrier<1, kSelThreads>;
@@ -75,9 +80,7 @@ struct Layout {
   // warp 0 and warps 2.. produce, warp 1 issues MMAs, then the selectors
   static constexpr int kFirstSel = kStages + 1;
   static constexpr int kThreads = 32 * kFirstSel + kSelThreads;
-  static constexpr uint32_t kQBytes = kBM * D * 2;
-  static constexpr size_t q_off = 0;
-  static constexpr size_t k_off = q_off + kQBytes;
+  static constexpr size_t k_off = 0;
   static constexpr size_t seg_off = k_off + (size_t)kStages * kStageBytes;
   // segments, or the pass-1 slot table (128 rows x 256 bf16) before them
   __host__ __device__ static size_t bytes(int P) {
@@ -106,6 +109,7 @@ struct Shared {
   unsigned char xcnt[kSelThreads];  // entries in the spare segment
   signed char xcol[kSelThreads];    // spare segment index, -1: none
   unsigned char ovf[kSelThreads];   // 1: candidates did not fit
+  float xsum[kSelThreads];          // per thread: candidates' sum (masses)
 };
 
 __device__ __forceinline__ int quad_sum(int v) {
@@ -258,8 +262,7 @@ __device__ __forceinline__ void quad_cut(const unsigned char* seg, int col_own,
 
 template <int D, bool MASS>
 __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
-prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
+prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
                       int P, int maps3d) {
   using Lay = Layout<D>;
   constexpr int KT = Lay::KT;
@@ -268,7 +271,6 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = smem + Lay::q_off;
   unsigned char* sK = smem + Lay::k_off;
   unsigned char* seg = smem + Lay::seg_off;
   __shared__ Shared sh;
@@ -286,7 +288,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       sm100::mbar_init(&sh.kfull[s], 1);
       sm100::mbar_init(&sh.kempty[s], 1);
     }
-    sm100::mbar_init(&sh.qfull, 1);
+    sm100::mbar_init(&sh.qfull, 4);  // the four Q-writing selector warps
     sm100::mbar_init(&sh.never, 1);
     for (int t = 0; t < kTmemBufs; ++t) {
       sm100::mbar_init(&sh.tfull[t], 1);
@@ -297,7 +299,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sm100::fence_barrier_init();
   }
   if (warp == 1) {
-    sm100::tmem_alloc(&sh.tmem, kTmemBufs * kBN);
+    sm100::tmem_alloc(&sh.tmem, 512);
     sm100::tmem_relinquish();
   }
   sm100::tc_fence_before();
@@ -317,18 +319,6 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     if (lane == 0 && T > 0) {
       sm100::prefetch_tmap(&tmK);
       const int krow = (b * a.Hkv + g) * a.L;
-      if (p == 0) {
-        sm100::prefetch_tmap(&tmQ);
-        const int qrow = (b * a.Hq + h) * a.nq + i0;
-        sm100::mbar_arrive_expect_tx(&sh.qfull, Lay::kQBytes);
-        if (D == 64 || !maps3d) {
-          for (int kb = 0; kb < D / 64; ++kb)
-            sm100::tma_load_2d(sQ + kb * kBlockBytes, &tmQ, &sh.qfull,
-                               kb * 64, qrow);
-        } else {
-          sm100::tma_load_3d(sQ, &tmQ, &sh.qfull, 0, qrow, 0);
-        }
-      }
       int last = -1;  // the last stage sequence index this producer issued
       for (int u = p; u < 2 * TS; u += kStages) {
         const int s = p;
@@ -352,7 +342,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         last = u;
       }
       // every copy this thread started must land before the CTA can exit
-      bool drained = p != 0 || sm100::mbar_wait(&sh.qfull, 0, kDrainWaitNs);
+      bool drained = true;
       if (last >= 0)
         drained &= sm100::mbar_wait(&sh.kfull[p], (last / kStages) & 1,
                                     kDrainWaitNs);
@@ -362,7 +352,6 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     // ---------------- MMA issuer
     if (lane == 0 && T > 0) {
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kBN);
-      const uint32_t aq = sm100::smem_u32(sQ);
       const uint32_t ak = sm100::smem_u32(sK);
       int tt = 0;  // accumulator tiles issued, both passes
       if (a.stall_ns) {
@@ -383,7 +372,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int q = 0; q < KT; ++q) {
             if (t0 + q >= T) break;
-            const int buf = tt & (kTmemBufs - 1);
+            const int buf = tt % kTmemBufs;
             if (tt >= kTmemBufs &&
                 !sm100::wait_or_abort(&sh.tempty[buf], ((tt / kTmemBufs) & 1) ^ 1,
                                       abort_flag, a.status, a.wait_ns)) {
@@ -396,9 +385,9 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-              sm100::mma_bf16(d_tmem, sm100::desc_k_sw128(aq + off),
-                              sm100::desc_k_sw128(kt + off), idesc,
-                              kk > 0 ? 1u : 0u);
+              sm100::mma_bf16_ts(d_tmem, tmem + kQCol + kk * 8,
+                                 sm100::desc_k_sw128(kt + off), idesc,
+                                 kk > 0 ? 1u : 0u);
             }
             sm100::mma_commit(&sh.tfull[buf]);
             ++tt;
@@ -408,7 +397,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       }
       // The last commit covers every MMA issued: wait for it before exit.
       if (tt > 0 &&
-          !sm100::mbar_wait(&sh.tfull[(tt - 1) & (kTmemBufs - 1)],
+          !sm100::mbar_wait(&sh.tfull[(tt - 1) % kTmemBufs],
                             ((tt - 1) / kTmemBufs) & 1, kDrainWaitNs))
         raise_flag(a.status, kErrTimeout);
     }
@@ -422,11 +411,38 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     const int hi = sh.hi[r];
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + grp * 32;
 
+    if (grp == 0) {
+      // the Q tile into TMEM columns kQCol..: this warp's 32 rows, each
+      // thread its own row as bf16 pairs (zeros past the last query row)
+      const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16) + kQCol;
+      const bool qv = i0 + r < a.nq;
+      const uint4* qp = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(a.Q) +
+          ((size_t)(b * a.Hq + h) * a.nq + (qv ? i0 + r : 0)) * D);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 v = qv ? qp[c * 8 + e] : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * e] = v.x;
+          w[4 * e + 1] = v.y;
+          w[4 * e + 2] = v.z;
+          w[4 * e + 3] = v.w;
+        }
+        sm100::tmem_st_32x32b_x32(tq + c * 32, w);
+      }
+      sm100::tmem_wait_st();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sh.qfull);
+    }
+
     // Scores of accumulator tile tt (key tile t of its pass) for this
     // thread's row and chunk, non-candidates (j = 0, the window, the future)
     // replaced by NaN.
     auto fetch = [&](int tt, int t, uint32_t (&raw)[32]) -> bool {
-      const int buf = tt & (kTmemBufs - 1);
+      const int buf = tt % kTmemBufs;
       if (!__all_sync(0xFFFFFFFFu,
                       sm100::wait_or_abort(&sh.tfull[buf], (tt / kTmemBufs) & 1,
                                            abort_flag, a.status, a.wait_ns)))
@@ -594,10 +610,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sh.xcnt[col] = (unsigned char)(xc < 0 ? 0 : last);
     sh.xcol[col] = (signed char)xc;
     sh.ovf[col] = ovf ? 1 : 0;
-    // per thread: sum of 2^((s - M) log2e/sqrt(d)) over its candidates, in
-    // the Q tile's bytes (every MMA reading them has completed: this thread
-    // consumed the last accumulator)
-    if constexpr (MASS) reinterpret_cast<float*>(sQ)[col] = xs;
+    // per thread: sum of 2^((s - M) log2e/sqrt(d)) over its candidates
+    if constexpr (MASS) sh.xsum[col] = xs;
     SelBar::sync();
     {
       // ---- exact Top-k per row: four lanes per row, eight rows per warp
@@ -612,7 +626,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       const size_t grow = (size_t)(b * a.Hq + h) * a.nq + rq;
       bool live = rq < a.nq;
       if constexpr (MASS) {
-        float t = reinterpret_cast<const float*>(sQ)[cown];
+        float t = sh.xsum[cown];
         t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
         t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
         if (live && part == 0)
@@ -641,74 +655,25 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   __syncthreads();
   if (warp == 1) {
     sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, kTmemBufs * kBN);
+    sm100::tmem_dealloc(tmem, 512);
   }
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
-                                &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// Row-major [rows, d] bf16 tensor read in boxes of `box_rows` rows x 64
-// columns with the 128-byte swizzle (the UMMA K-major SW128 layout).
-bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, int d,
-                  int box_rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  if (d != 64) dims[0] = (cuuint64_t)d;
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The same [rows, 128] tensor seen as (64 columns, rows, 2 column halves),
-// so that one box of 128 rows x both halves lands as the two 16 KB
-// column-half blocks of the SW128 layout in a single 32 KB copy.
-bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {64, (cuuint64_t)rows, 2};
-  cuuint64_t strides[2] = {256, 128};
-  cuuint32_t box[3] = {64, 128, 2};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
-             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_d(const PrefillArgs& a, cudaStream_t s) {
   using Lay = Layout<D>;
-  CUtensorMap tq, tk;
+  CUtensorMap tk;
   int maps3d = 0;
-  const uint64_t qrows = (uint64_t)a.B * a.Hq * a.nq;
   const uint64_t krows = (uint64_t)a.B * a.Hkv * a.L;
   if (D == 64) {
-    if (!make_tmap_2d(&tq, a.Q, qrows, D, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&tk, a.K, krows, D, kBN * Lay::KT))
       return cudaErrorInvalidValue;
-  } else if (make_tmap_3d(&tq, a.Q, qrows) && make_tmap_3d(&tk, a.K, krows)) {
+  } else if (make_tmap_3d(&tk, a.K, krows, kBN)) {
     maps3d = 1;
-  } else {
+  } else if (!make_tmap_2d(&tk, a.K, krows, D, kBN)) {
     // two 16 KB copies per stage when the 3-D view is refused
-    if (!make_tmap_2d(&tq, a.Q, qrows, D, kBM)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tk, a.K, krows, D, kBN)) return cudaErrorInvalidValue;
+    return cudaErrorInvalidValue;
   }
   // Segment positions per (row, chunk group) thread: about k/4 entries are
   // expected (about 1.1 k per row), with the spare segments for the rest.
@@ -725,7 +690,7 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   dim3 grid((a.nq + kBM - 1) / kBM, a.Hq, a.B);
   prof_before(s, "prefill_score_topk_tc");
-  kern<<<grid, Lay::kThreads, smem, s>>>(tq, tk, a, P, maps3d);
+  kern<<<grid, Lay::kThreads, smem, s>>>(tk, a, P, maps3d);
   prof_after(s);
   return cudaGetLastError();
 }

@@ -110,4 +110,77 @@ __device__ void cta_select_thresholds(const uint64_t* keys, int stride,
   Bar::sync();
 }
 
+// One warp cuts the list lst[0..n) of unique keys down to its best kk keys
+// (n > kk >= 1), in place and in no particular order, and returns the
+// threshold T with exactly kk keys >= T.  Radix select from the most
+// significant byte, stopping as soon as the chosen byte's bucket holds
+// exactly the keys still needed (its lower bound then separates the sets).
+__device__ __forceinline__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint32_t* hist,
+                             int lane) {
+  uint64_t prefix = 0ull;
+  uint32_t need = (uint32_t)kk;
+#pragma unroll 1
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    const uint64_t hmask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
+#pragma unroll
+    for (int b = lane; b < 256; b += 32) hist[b] = 0u;
+    __syncwarp();
+    for (int e = lane; e < n; e += 32) {
+      const uint64_t key = lst[e];
+      if ((key & hmask) == prefix)
+        atomicAdd(&hist[(uint32_t)(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      c[t] = hist[255 - 8 * lane - t];
+      sum += c[t];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const bool mine = excl < need && need <= incl;
+    uint32_t digit = 0, nd = 0, bucket = 0;
+    if (mine) {
+      uint32_t acc = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (acc + c[t] >= need) {
+          digit = 255u - 8u * lane - t;
+          nd = need - acc;
+          bucket = c[t];
+          break;
+        }
+        acc += c[t];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
+    nd = __shfl_sync(0xFFFFFFFFu, nd, src);
+    bucket = __shfl_sync(0xFFFFFFFFu, bucket, src);
+    prefix |= (uint64_t)digit << shift;
+    need = nd;
+    __syncwarp();  // the histogram is cleared again next pass
+    if (bucket == nd) break;
+  }
+  // keep the keys >= prefix, packed to the front in reading order; a slot
+  // is only written after the whole group of 32 that covers it was read
+  int wr = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int e = base + lane;
+    const uint64_t key = e < n ? lst[e] : 0ull;
+    const bool keep = e < n && key >= prefix;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) lst[wr + __popc(bal & ((1u << lane) - 1u))] = key;
+    wr += __popc(bal);
+    __syncwarp();
+  }
+  return prefix;
+}
+
 }  // namespace ca
