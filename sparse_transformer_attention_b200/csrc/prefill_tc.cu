@@ -600,10 +600,15 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
           xs += exp2f(fmaxf((__uint_as_float(raw[x]) - Mr) * sl2, -INFINITY));
       }
       const int j0 = t * kBN + grp * 32;
+      static_assert(32 % kCheck == 0 && 32 / kCheck == 4, "four runs");
       room();
       append_run<0>(raw, cur, ovf ? INFINITY : Lr, j0);
       room();
       append_run<kCheck>(raw, cur, ovf ? INFINITY : Lr, j0);
+      room();
+      append_run<2 * kCheck>(raw, cur, ovf ? INFINITY : Lr, j0);
+      room();
+      append_run<3 * kCheck>(raw, cur, ovf ? INFINITY : Lr, j0);
     }
     const int last = (cur - base) / kEntStride;
     sh.cnt[col] = (unsigned char)(xc < 0 ? last : own);
