@@ -547,24 +547,56 @@ __device__ __forceinline__ uint32_t bf16_bits_as_f32(const __nv_bfloat16* p) {
 
 constexpr int kMmaWarps = 4;  // 16 query rows each
 
-// Per warp: the window state (o, max, sum) of its 16 rows, then their Top-k
-// keys as loaded in step 1.
+// Shared memory of the bf16 gather: the Top-k keys of every warp's 16 rows
+// (kept to the end), then the window's K and V rows staged in chunks of 64
+// keys (two buffers, rows padded by 16 bytes so that the fragment loads of
+// eight rows fall on different banks).  After the window phase the staging
+// bytes hold each warp's window state (o, max, sums) instead.
 template <int D>
 struct MmaGatherSmem {
+  static constexpr int CK = 64;                 // keys per staged chunk
+  static constexpr int RS = D * 2 + 16;         // padded row stride (bytes)
+  static constexpr size_t chunk = (size_t)CK * RS;
+  static constexpr size_t stage = 4 * chunk;    // two buffers of K and V
   static constexpr size_t state = (size_t)16 * D * 4 + 3 * 16 * 4;
-  __host__ __device__ static size_t per_warp(int k) {
-    return state + (size_t)16 * k * 8;
+  static_assert(stage >= kMmaWarps * state, "window state fits the staging");
+  __host__ __device__ static size_t keys(int k) {
+    return (size_t)kMmaWarps * 16 * k * 8;
   }
-  __host__ __device__ static size_t bytes(int k) { return kMmaWarps * per_warp(k); }
+  __host__ __device__ static size_t bytes(int k) { return keys(k) + stage; }
 };
 
-// bf16 gather with the window on tensor cores.  A warp owns 16 consecutive
-// query rows of one (batch, head).
-//   1. The Top-k keys of its rows into shared memory in one batch of loads,
-//      then C_i and |C_i| for each row (whole warp per row).
-//   2. The window [lo_i, i] of all 16 rows: MMA scores, masked per row, an
-//      online softmax per row over 16-key blocks, and the MMA p * V.  The
-//      state (max, sum, unnormalised o) goes to shared memory.
+__device__ __forceinline__ uint32_t lds32(const unsigned char* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+__device__ __forceinline__ uint32_t lds_bf16_as_f32(const unsigned char* p) {
+  return (uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16;
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// bf16 gather with the window on tensor cores.  A CTA owns 64 consecutive
+// query rows of one (batch, head), a warp 16 of them.
+//   1. The Top-k keys of the warp's rows into shared memory in one batch of
+//      loads, then C_i and |C_i| for each row (whole warp per row).
+//   2. The window [lo_i, i] of all rows: the CTA stages the K and V rows of
+//      the window span in 64-key chunks (16-byte asynchronous copies, the
+//      next chunk in flight while the current one is used); each warp runs
+//      its rows over the 16-key blocks it needs: MMA scores, masked per row,
+//      an online softmax per row, and the MMA p * V, with every fragment
+//      read from shared memory.  The state (max, sum, unnormalised o) then
+//      goes to shared memory.
 //   3. Eight lanes per row, four rows at a time: start from the window state
 //      and fold in the Top-k keys (scores from the selector) and the anchor
 //      (score computed here), then write the output row.
@@ -572,27 +604,35 @@ template <int D, typename TO, int NPL, bool MASS>
 __global__ void __launch_bounds__(kMmaWarps * 32)
 prefill_gather_mma(PrefillArgs a) {
   using T = __nv_bfloat16;
+  using SM = MmaGatherSmem<D>;
   constexpr int KS = D / 16;  // k-steps of the score MMA
   constexpr int NT = D / 8;   // head-dim tiles of the p * V MMA
+  constexpr int RS = SM::RS;
   extern __shared__ __align__(16) unsigned char g_smem[];
+  __shared__ int s_kmin;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   // query rows r at positions p0 + r, keys 0..L-1
   const int nq = a.nq, L = a.L, p0 = a.p0, k = a.k;
-  float* s_o = reinterpret_cast<float*>(g_smem + wid * MmaGatherSmem<D>::per_warp(k));
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(g_smem) + (size_t)wid * 16 * k;
+  unsigned char* stage = g_smem + SM::keys(k);
+  float* s_o = reinterpret_cast<float*>(stage + wid * SM::state);
   float* s_m = s_o + 16 * D;
   float* s_l = s_m + 16;
   float* s_lx = s_l + 16;  // window sums of the unrounded weights (reports)
-  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_lx + 16);  // [16][k]
   const int bh = blockIdx.y;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const int i0 = (blockIdx.x * kMmaWarps + wid) * 16;  // first query row
-  if (i0 >= nq) return;  // the whole warp
+  const int r0 = blockIdx.x * kMmaWarps * 16;  // first query row of the CTA
+  const int i0 = r0 + wid * 16;                // first query row of the warp
+  const bool wlive = i0 < nq;  // every warp takes part in the staging
   const int64_t rowbase = (int64_t)bh * nq;
   const T* Qg = reinterpret_cast<const T*>(a.Q) + rowbase * D;
   const T* Kg = reinterpret_cast<const T*>(a.K) + ((size_t)b * a.Hkv + g) * (size_t)L * D;
   const T* Vg = reinterpret_cast<const T*>(a.V) + ((size_t)b * a.Hkv + g) * (size_t)L * D;
+  if (threadIdx.x == 0) s_kmin = 0x7FFFFFFF;
+  __syncthreads();
 
+  if (wlive) {
   // ---- 1: the Top-k keys of the warp's rows (16 consecutive rows of one
   // head: one contiguous run) into shared memory, 16 loads in flight per
   // lane, then C_i one row at a time across the warp
@@ -635,6 +675,8 @@ prefill_gather_mma(PrefillArgs a) {
     write_set<NPL>(a, rowbase + r, v, m, i, lo, lane);
   }
 
+  }  // wlive
+
   // ---- 2: window on tensor cores
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);
   const int gr = lane >> 2, tq = lane & 3;  // fragment row group, thread in group
@@ -653,6 +695,7 @@ prefill_gather_mma(PrefillArgs a) {
   for (int off = 16; off > 0; off >>= 1)
     kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, off));
   const int kmax = p0 + min(i0 + 15, nq - 1);
+  if (wlive && lane == 0) atomicMin(&s_kmin, kmin);
   uint32_t qa[KS][4];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
@@ -668,82 +711,117 @@ prefill_gather_mma(PrefillArgs a) {
 #pragma unroll
   for (int nd = 0; nd < NT; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
 
+  // the CTA's window span, staged in chunks of SM::CK keys starting at a
+  // multiple of 16 (a 16-key block never straddles two chunks)
+  __syncthreads();
+  const int cs0 = s_kmin & ~15;
+  const int kmax_c = p0 + min(r0 + kMmaWarps * 16 - 1, nq - 1);
+  const int nch = (kmax_c - cs0) / SM::CK + 1;
+  auto stage_chunk = [&](int m) {
+    unsigned char* dK = stage + (m & 1) * 2 * SM::chunk;
+    unsigned char* dV = dK + SM::chunk;
+    const int cs = cs0 + m * SM::CK;
+    constexpr int kPieces = D * 2 / 16;  // 16-byte pieces per row
+    for (int e = threadIdx.x; e < SM::CK * kPieces; e += kMmaWarps * 32) {
+      const int rr = e / kPieces, pc = e % kPieces;
+      const int j = min(cs + rr, L - 1);  // rows past the cache: any valid
+      cp_async16(dK + rr * RS + pc * 16, Kg + (size_t)j * D + pc * 8);
+      cp_async16(dV + rr * RS + pc * 16, Vg + (size_t)j * D + pc * 8);
+    }
+    cp_async_commit();
+  };
+  stage_chunk(0);
 #pragma unroll 1
-  for (int j0 = kmin & ~15; j0 <= kmax; j0 += 16) {
-    float s[2][4];
-#pragma unroll
-    for (int h8 = 0; h8 < 2; ++h8) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int krow = min(j0 + 8 * h8 + gr, L - 1);
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int c = 16 * ks + 2 * tq;
-        mma_bf16_16816(acc, qa[ks], ld_b32(Kg + (size_t)krow * D + c),
-                       ld_b32(Kg + (size_t)krow * D + c + 8));
-      }
-      const int kc = j0 + 8 * h8 + 2 * tq;  // key of acc[0] / acc[2]
-      s[h8][0] = (va && kc >= loa && kc <= ia) ? acc[0] * sl2 : -INFINITY;
-      s[h8][1] = (va && kc + 1 >= loa && kc + 1 <= ia) ? acc[1] * sl2 : -INFINITY;
-      s[h8][2] = (vb && kc >= lob && kc <= ib) ? acc[2] * sl2 : -INFINITY;
-      s[h8][3] = (vb && kc + 1 >= lob && kc + 1 <= ib) ? acc[3] * sl2 : -INFINITY;
+  for (int m = 0; m < nch; ++m) {
+    if (m + 1 < nch) {
+      stage_chunk(m + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    float xa = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-    float xb = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-    xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 1));
-    xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 2));
-    xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 1));
-    xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 2));
-    const float na = fmaxf(ma, xa), nb = fmaxf(mb, xb);
-    const float sa = na == -INFINITY ? 1.f : exp2f(ma - na);
-    const float sb = nb == -INFINITY ? 1.f : exp2f(mb - nb);
-    la *= sa;
-    lb *= sb;
-    if constexpr (MASS) {
-      lax *= sa;
-      lbx *= sb;
+    __syncthreads();
+    const int cs = cs0 + m * SM::CK;
+    const unsigned char* sK = stage + (m & 1) * 2 * SM::chunk;
+    const unsigned char* sV = sK + SM::chunk;
+    const int jlo = max(cs, kmin & ~15), jhi = min(cs + SM::CK - 1, kmax);
+#pragma unroll 1
+    for (int j0 = jlo; wlive && j0 <= jhi; j0 += 16) {
+        float s[2][4];
+    #pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          const unsigned char* kr = sK + (j0 - cs + 8 * h8 + gr) * RS;
+    #pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const int c = 16 * ks + 2 * tq;
+            mma_bf16_16816(acc, qa[ks], lds32(kr + c * 2), lds32(kr + c * 2 + 16));
+          }
+          const int kc = j0 + 8 * h8 + 2 * tq;  // key of acc[0] / acc[2]
+          s[h8][0] = (va && kc >= loa && kc <= ia) ? acc[0] * sl2 : -INFINITY;
+          s[h8][1] = (va && kc + 1 >= loa && kc + 1 <= ia) ? acc[1] * sl2 : -INFINITY;
+          s[h8][2] = (vb && kc >= lob && kc <= ib) ? acc[2] * sl2 : -INFINITY;
+          s[h8][3] = (vb && kc + 1 >= lob && kc + 1 <= ib) ? acc[3] * sl2 : -INFINITY;
+        }
+        float xa = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        float xb = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 1));
+        xa = fmaxf(xa, __shfl_xor_sync(0xFFFFFFFFu, xa, 2));
+        xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 1));
+        xb = fmaxf(xb, __shfl_xor_sync(0xFFFFFFFFu, xb, 2));
+        const float na = fmaxf(ma, xa), nb = fmaxf(mb, xb);
+        const float sa = na == -INFINITY ? 1.f : exp2f(ma - na);
+        const float sb = nb == -INFINITY ? 1.f : exp2f(mb - nb);
+        la *= sa;
+        lb *= sb;
+        if constexpr (MASS) {
+          lax *= sa;
+          lbx *= sb;
+        }
+    #pragma unroll
+        for (int nd = 0; nd < NT; ++nd) {
+          o[nd][0] *= sa;
+          o[nd][1] *= sa;
+          o[nd][2] *= sb;
+          o[nd][3] *= sb;
+        }
+        uint32_t p[2][4];
+    #pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const float p0 = s[h8][0] == -INFINITY ? 0.f : exp2f(s[h8][0] - na);
+          const float p1 = s[h8][1] == -INFINITY ? 0.f : exp2f(s[h8][1] - na);
+          const float p2 = s[h8][2] == -INFINITY ? 0.f : exp2f(s[h8][2] - nb);
+          const float p3 = s[h8][3] == -INFINITY ? 0.f : exp2f(s[h8][3] - nb);
+          p[h8][0] = to_tf32(p0);
+          p[h8][1] = to_tf32(p1);
+          p[h8][2] = to_tf32(p2);
+          p[h8][3] = to_tf32(p3);
+          // the sums use the rounded weights, as the MMA does
+          la += __uint_as_float(p[h8][0]) + __uint_as_float(p[h8][1]);
+          lb += __uint_as_float(p[h8][2]) + __uint_as_float(p[h8][3]);
+          if constexpr (MASS) {
+            lax += p0 + p1;
+            lbx += p2 + p3;
+          }
+        }
+        // p * V, keys of the k8 step ordered (2t, 2t+1) -> (t, t+4) so that the
+        // score fragment is the A fragment as it stands
+    #pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const unsigned char* v0r = sV + (j0 - cs + 8 * h8 + 2 * tq) * RS;
+          const unsigned char* v1r = v0r + RS;
+    #pragma unroll
+          for (int nd = 0; nd < NT; ++nd) {
+            const uint32_t b0 = lds_bf16_as_f32(v0r + (8 * nd + gr) * 2);
+            const uint32_t b1 = lds_bf16_as_f32(v1r + (8 * nd + gr) * 2);
+            mma_tf32_1688(o[nd], p[h8][0], p[h8][2], p[h8][1], p[h8][3], b0, b1);
+          }
+        }
+        ma = na;
+        mb = nb;
     }
-#pragma unroll
-    for (int nd = 0; nd < NT; ++nd) {
-      o[nd][0] *= sa;
-      o[nd][1] *= sa;
-      o[nd][2] *= sb;
-      o[nd][3] *= sb;
-    }
-    uint32_t p[2][4];
-#pragma unroll
-    for (int h8 = 0; h8 < 2; ++h8) {
-      const float p0 = s[h8][0] == -INFINITY ? 0.f : exp2f(s[h8][0] - na);
-      const float p1 = s[h8][1] == -INFINITY ? 0.f : exp2f(s[h8][1] - na);
-      const float p2 = s[h8][2] == -INFINITY ? 0.f : exp2f(s[h8][2] - nb);
-      const float p3 = s[h8][3] == -INFINITY ? 0.f : exp2f(s[h8][3] - nb);
-      p[h8][0] = to_tf32(p0);
-      p[h8][1] = to_tf32(p1);
-      p[h8][2] = to_tf32(p2);
-      p[h8][3] = to_tf32(p3);
-      // the sums use the rounded weights, as the MMA does
-      la += __uint_as_float(p[h8][0]) + __uint_as_float(p[h8][1]);
-      lb += __uint_as_float(p[h8][2]) + __uint_as_float(p[h8][3]);
-      if constexpr (MASS) {
-        lax += p0 + p1;
-        lbx += p2 + p3;
-      }
-    }
-    // p * V, keys of the k8 step ordered (2t, 2t+1) -> (t, t+4) so that the
-    // score fragment is the A fragment as it stands
-#pragma unroll
-    for (int h8 = 0; h8 < 2; ++h8) {
-      const int kv0 = min(j0 + 8 * h8 + 2 * tq, L - 1);
-      const int kv1 = min(j0 + 8 * h8 + 2 * tq + 1, L - 1);
-#pragma unroll
-      for (int nd = 0; nd < NT; ++nd) {
-        const uint32_t b0 = bf16_bits_as_f32(Vg + (size_t)kv0 * D + 8 * nd + gr);
-        const uint32_t b1 = bf16_bits_as_f32(Vg + (size_t)kv1 * D + 8 * nd + gr);
-        mma_tf32_1688(o[nd], p[h8][0], p[h8][2], p[h8][1], p[h8][3], b0, b1);
-      }
-    }
-    ma = na;
-    mb = nb;
+    __syncthreads();  // the next chunk overwrites this buffer
   }
+  if (!wlive) return;
   la += __shfl_xor_sync(0xFFFFFFFFu, la, 1);
   la += __shfl_xor_sync(0xFFFFFFFFu, la, 2);
   lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 1);
