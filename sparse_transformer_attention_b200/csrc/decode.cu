@@ -525,6 +525,29 @@ decode_merge_attend(DecodeArgs a) {
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
+    // every list into shared memory at once: 16-byte asynchronous copies
+    // (the list area of a head starts 16-byte aligned: k keys per chunk,
+    // 8 bytes each, and the workspace lists start at a 256-byte boundary;
+    // an odd k leaves the head's area 8-byte aligned: then plain loads)
+    if ((((uintptr_t)src) & 15u) == 0) {
+      for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         (uint32_t)__cvta_generic_to_shared(cand + e)),
+                     "l"(src + e)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    } else {
+      for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
+    }
+    if (gtid == 0) {
+      s_n = 0;
+      s_m = 0;
+      s_kk = m > 0 ? m : 1;
+    }
+    MergeBar::sync();
     // Every chunk list holds its chunk's best k keys, so the largest of the
     // lists' smallest keys, T0, is at most the global k-th best key (the
     // chunk that has it alone holds k keys >= T0): only keys >= T0 can be
@@ -533,27 +556,26 @@ decode_merge_attend(DecodeArgs a) {
     uint64_t t0 = 0ull;
     for (int c = gw; c < a.nchunks; c += 8) {
       uint64_t mn = ~0ull;
-      for (int e = lane; e < kh; e += 32) mn = min(mn, src[(size_t)c * k + e]);
+      for (int e = lane; e < kh; e += 32) mn = min(mn, cand[(size_t)c * k + e]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
         mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
       t0 = max(t0, mn);
     }
     if (lane == 0) s_t0[gw] = t0;
-    if (gtid == 0) {
-      s_n = 0;
-      s_m = 0;
-      s_kk = m > 0 ? m : 1;
-    }
     MergeBar::sync();
     t0 = s_t0[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) t0 = max(t0, s_t0[w]);
-    // keep the keys >= T0 (and real), packed to the front in any order
+    // keep the keys >= T0 (and real), packed to the front in any order: in
+    // place, one round of 256 keys at a time (a round's keys are all read
+    // before any of them is written, and the kept count never passes the
+    // keys read so far)
     for (int e0 = 0; e0 < ncand; e0 += 256) {
       const int e = e0 + gtid;
-      const uint64_t key = e < ncand ? src[e] : 0ull;
+      const uint64_t key = e < ncand ? cand[e] : 0ull;
       const bool keep = key != 0ull && key >= t0;
+      MergeBar::sync();
       const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
       int base = 0;
       if (lane == 0 && bal) base = atomicAdd(&s_n, __popc(bal));

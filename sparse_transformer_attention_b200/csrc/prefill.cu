@@ -541,9 +541,6 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
 __device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16* p) {
   return __ldg(reinterpret_cast<const unsigned int*>(p));
 }
-__device__ __forceinline__ uint32_t bf16_bits_as_f32(const __nv_bfloat16* p) {
-  return (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16;
-}
 
 constexpr int kMmaWarps = 4;  // 16 query rows each
 
