@@ -183,10 +183,12 @@ CA_API ca_status condensate_attn_decode(const void* q, const void* K, const void
                                  void* stream);
 
 /*
- * Number of key chunks the decode score pass splits an L-long cache into on
- * the current device (about two CTAs per SM).  The decode workspace holds,
- * after its 256-byte status area, the best k selection keys of every chunk
- * and q-head, [B, Hq, chunks, k] 64-bit keys (fp32 score bits in an
+ * Number of workers (CTAs per batch and kv-head) of the decode score pass on
+ * the current device (about two CTAs per SM); each keeps one candidate list
+ * per q-head over the part of the cache it streamed.  The decode workspace
+ * holds, after its 256-byte status area and a 256-byte-rounded area of
+ * B * Hkv 32-bit work counters, the best k selection keys of every worker
+ * and q-head, [B, Hq, workers, k] 64-bit keys (fp32 score bits in an
  * order-preserving form in the high word, 0xFFFFFFFF - position in the low
  * word, 0 for an empty slot), in a 256-byte-rounded area.  For tests and
  * debugging; 0 for invalid sizes.

@@ -30,14 +30,20 @@ bool group_ok(int Hq, int Hkv) {
   return G == 1 || G == 2 || G == 4 || G == 8;
 }
 
-// Decode workspace: status area | chunk lists [B, Hq, chunks, k] (64-bit
-// keys) | per-chunk candidate (max, sum) [B, Hq, chunks] (float2).
+// Decode workspace: status area | unit counters [B, Hkv] (int32) | worker
+// lists [B, Hq, workers, k] (64-bit keys) | per-worker candidate (max, sum)
+// [B, Hq, workers] (float2).  The status area and the counters are cleared
+// by each call.
+size_t decode_claims_bytes(int B, int Hkv) {
+  return round_up((size_t)B * Hkv * 4, 256);
+}
 size_t decode_lists_bytes(int B, int Hq, int nch, int k) {
   return round_up((size_t)B * Hq * nch * (k > 0 ? k : 1) * 8, 256);
 }
 size_t decode_ws(int B, int L, int Hq, int Hkv, int k) {
   const int nch = ca::decode_chunks(B, L, Hkv, k);
-  return ca::kStatusBytes + decode_lists_bytes(B, Hq, nch, k) +
+  return ca::kStatusBytes + decode_claims_bytes(B, Hkv) +
+         decode_lists_bytes(B, Hq, nch, k) +
          round_up((size_t)B * Hq * nch * 8, 256);
 }
 
@@ -145,7 +151,8 @@ ca_status condensate_attn_decode_ex(const void* q, const void* K,
   if (k > ca::kDecodeMaxK) return CA_ERR_UNSUPPORTED;
   if (workspace_bytes < decode_ws(B, L, Hq, Hkv, k)) return CA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemsetAsync(workspace, 0, ca::kStatusBytes, s) != cudaSuccess)
+  const size_t cleared = ca::kStatusBytes + decode_claims_bytes(B, Hkv);
+  if (cudaMemsetAsync(workspace, 0, cleared, s) != cudaSuccess)
     return CA_ERR_CUDA;
   ca::DecodeArgs a;
   a.q = q; a.K = K; a.V = V;
@@ -157,7 +164,8 @@ ca_status condensate_attn_decode_ex(const void* q, const void* K,
   a.chunk_len = ca::decode_chunk_len(L, a.nchunks);
   a.kpow2 = next_pow2(k > 1 ? k : 2);
   a.status = (uint32_t*)workspace;
-  a.cand = (uint64_t*)((char*)workspace + ca::kStatusBytes);
+  a.claims = (int*)((char*)workspace + ca::kStatusBytes);
+  a.cand = (uint64_t*)((char*)workspace + cleared);
   a.cand_ml = (float2*)((char*)a.cand +
                         decode_lists_bytes(B, Hq, a.nchunks, k));
   a.wait_ns = ca::kPipelineWaitNs;

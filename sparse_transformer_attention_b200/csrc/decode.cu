@@ -430,6 +430,66 @@ struct Online {
   }
 };
 
+// Merge, first level: warp gw keeps the best kh of its share of the
+// q-head's ncand worker keys (read from global memory straight into
+// registers) and appends them to lvl at an offset taken from *s_n.
+template <int NPL>
+__device__ __forceinline__ void merge_level1(const uint64_t* src, int n,
+                                             int kh, uint64_t* lvl, int* s_n,
+                                             int lane) {
+  uint64_t v[NPL];
+  warp_load_keys<NPL>(src, n, v, lane);
+  const uint64_t T = warp_kth<NPL>(v, kh);
+  uint32_t cnt = 0u;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) cnt += v[t] >= T;
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  int base = 0;
+  if (lane == 0 && cnt) base = atomicAdd(s_n, (int)cnt);
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  warp_keep<NPL>(v, T, lvl + base, lane);
+}
+
+// Merge, second level (one warp): the best m (1 <= m <= 128) of the n
+// first-level keys in lvl, written as (position, score) pairs in ascending
+// position order to topj/tops[0..); returns how many were selected.  lvl is
+// reused as scratch.
+template <int NPL>
+__device__ __forceinline__ int merge_level2(uint64_t* lvl, int n, int m,
+                                            uint32_t* topj, float* tops,
+                                            int lane) {
+  uint64_t v[NPL];
+  warp_load_keys<NPL>(lvl, n, v, lane);
+  const uint64_t T = warp_kth<NPL>(v, m);
+  // the selected keys as (position << 32 | score bits), packed to lvl[0..)
+#pragma unroll
+  for (int t = 0; t < NPL; ++t)
+    if (v[t] >= T)
+      v[t] = ((uint64_t)key_index(v[t]) << 32) |
+             __float_as_uint(key_score(v[t]));
+    else
+      v[t] = 0ull;
+  __syncwarp();
+  const int got = warp_keep<NPL>(v, 1ull, lvl, lane);
+  __syncwarp();
+  uint64_t srt[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int e = t * 32 + lane;
+    srt[t] = e < got && e < 128 ? lvl[e] : ~0ull;
+  }
+  warp_bitonic64<4>(srt, lane);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int e = t * 32 + lane;
+    if (e < got && e < 128) {
+      topj[e] = (uint32_t)(srt[t] >> 32);
+      tops[e] = __uint_as_float((uint32_t)srt[t]);
+    }
+  }
+  return got;
+}
+
 template <typename T, int D, typename TO>
 __global__ void __launch_bounds__(kMergeThreads)
 decode_merge_attend(DecodeArgs a) {
@@ -525,77 +585,107 @@ decode_merge_attend(DecodeArgs a) {
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
-    // every list into shared memory at once: 16-byte asynchronous copies
-    // (the list area of a head starts 16-byte aligned: k keys per chunk,
-    // 8 bytes each, and the workspace lists start at a 256-byte boundary;
-    // an odd k leaves the head's area 8-byte aligned: then plain loads)
-    if ((((uintptr_t)src) & 15u) == 0) {
-      for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                         (uint32_t)__cvta_generic_to_shared(cand + e)),
-                     "l"(src + e)
-                     : "memory");
+    if (a.kpow2 <= 128) {
+      // Two levels of register-resident selection: each warp keeps the best
+      // m of an eighth of the keys, then warp 0 the best m of those (at most
+      // 8 m <= 1024 keys), written in ascending position order.
+      if (gtid == 0) {
+        s_n = 0;
+        s_m = 0;
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    } else {
-      for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
-    }
-    if (gtid == 0) {
-      s_n = 0;
-      s_m = 0;
-      s_kk = m > 0 ? m : 1;
-    }
-    MergeBar::sync();
-    // Every chunk list holds its chunk's best k keys, so the largest of the
-    // lists' smallest keys, T0, is at most the global k-th best key (the
-    // chunk that has it alone holds k keys >= T0): only keys >= T0 can be
-    // selected.  A list of a chunk with fewer than k candidates has empty
-    // (0) slots and contributes 0.
-    uint64_t t0 = 0ull;
-    for (int c = gw; c < a.nchunks; c += 8) {
-      uint64_t mn = ~0ull;
-      for (int e = lane; e < kh; e += 32) mn = min(mn, cand[(size_t)c * k + e]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
-      t0 = max(t0, mn);
-    }
-    if (lane == 0) s_t0[gw] = t0;
-    MergeBar::sync();
-    t0 = s_t0[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) t0 = max(t0, s_t0[w]);
-    // keep the keys >= T0 (and real), packed to the front in any order: in
-    // place, one round of 256 keys at a time (a round's keys are all read
-    // before any of them is written, and the kept count never passes the
-    // keys read so far)
-    for (int e0 = 0; e0 < ncand; e0 += 256) {
-      const int e = e0 + gtid;
-      const uint64_t key = e < ncand ? cand[e] : 0ull;
-      const bool keep = key != 0ull && key >= t0;
       MergeBar::sync();
-      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-      int base = 0;
-      if (lane == 0 && bal) base = atomicAdd(&s_n, __popc(bal));
-      base = __shfl_sync(0xFFFFFFFFu, base, 0);
-      if (keep) cand[base + __popc(bal & ((1u << lane) - 1u))] = key;
-    }
-    MergeBar::sync();
-    cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
-                                            gtid);
-    if (m > 0) {
-      for (int e = gtid; e < s_n; e += 256) {
-        const uint64_t key = cand[e];
-        if (key >= s_T && key != 0ull) {
-          const uint32_t j = key_index(key);
-          const int p = atomicAdd(&s_m, 1);
-          if (p < m && j >= 1 && (int64_t)j <= i - Wb) {
-            topj[p] = j;
-            tops[p] = key_score(key);
-          } else {
-            raise_flag(a.status, kErrInternal);
+      if (m > 0) {
+        const int per = (ncand + 7) / 8;
+        const int beg = min(ncand, gw * per);
+        const int cnt = min(ncand - beg, per);
+        if (per <= 128) merge_level1<4>(src + beg, cnt, m, cand, &s_n, lane);
+        else if (per <= 256) merge_level1<8>(src + beg, cnt, m, cand, &s_n, lane);
+        else if (per <= 512) merge_level1<16>(src + beg, cnt, m, cand, &s_n, lane);
+        else merge_level1<32>(src + beg, cnt, m, cand, &s_n, lane);
+      }
+      MergeBar::sync();
+      if (m > 0 && gw == 0) {
+        const int n = s_n;
+        int got;
+        if (n <= 128) got = merge_level2<4>(cand, n, m, topj, tops, lane);
+        else if (n <= 256) got = merge_level2<8>(cand, n, m, topj, tops, lane);
+        else if (n <= 512) got = merge_level2<16>(cand, n, m, topj, tops, lane);
+        else got = merge_level2<32>(cand, n, m, topj, tops, lane);
+        if (lane == 0) s_m = got;
+      }
+    } else {
+      // every list into shared memory at once: 16-byte asynchronous copies
+      // (the list area of a head starts 16-byte aligned: k keys per chunk,
+      // 8 bytes each, and the workspace lists start at a 256-byte boundary;
+      // an odd k leaves the head's area 8-byte aligned: then plain loads)
+      if ((((uintptr_t)src) & 15u) == 0) {
+        for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                           (uint32_t)__cvta_generic_to_shared(cand + e)),
+                       "l"(src + e)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      } else {
+        for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
+      }
+      if (gtid == 0) {
+        s_n = 0;
+        s_m = 0;
+        s_kk = m > 0 ? m : 1;
+      }
+      MergeBar::sync();
+      // Every chunk list holds its chunk's best k keys, so the largest of the
+      // lists' smallest keys, T0, is at most the global k-th best key (the
+      // chunk that has it alone holds k keys >= T0): only keys >= T0 can be
+      // selected.  A list of a chunk with fewer than k candidates has empty
+      // (0) slots and contributes 0.
+      uint64_t t0 = 0ull;
+      for (int c = gw; c < a.nchunks; c += 8) {
+        uint64_t mn = ~0ull;
+        for (int e = lane; e < kh; e += 32) mn = min(mn, cand[(size_t)c * k + e]);
+  #pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+        t0 = max(t0, mn);
+      }
+      if (lane == 0) s_t0[gw] = t0;
+      MergeBar::sync();
+      t0 = s_t0[0];
+  #pragma unroll
+      for (int w = 1; w < 8; ++w) t0 = max(t0, s_t0[w]);
+      // keep the keys >= T0 (and real), packed to the front in any order: in
+      // place, one round of 256 keys at a time (a round's keys are all read
+      // before any of them is written, and the kept count never passes the
+      // keys read so far)
+      for (int e0 = 0; e0 < ncand; e0 += 256) {
+        const int e = e0 + gtid;
+        const uint64_t key = e < ncand ? cand[e] : 0ull;
+        const bool keep = key != 0ull && key >= t0;
+        MergeBar::sync();
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&s_n, __popc(bal));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        if (keep) cand[base + __popc(bal & ((1u << lane) - 1u))] = key;
+      }
+      MergeBar::sync();
+      cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
+                                              gtid);
+      if (m > 0) {
+        for (int e = gtid; e < s_n; e += 256) {
+          const uint64_t key = cand[e];
+          if (key >= s_T && key != 0ull) {
+            const uint32_t j = key_index(key);
+            const int p = atomicAdd(&s_m, 1);
+            if (p < m && j >= 1 && (int64_t)j <= i - Wb) {
+              topj[p] = j;
+              tops[p] = key_score(key);
+            } else {
+              raise_flag(a.status, kErrInternal);
+            }
           }
         }
       }
@@ -630,7 +720,8 @@ decode_merge_attend(DecodeArgs a) {
   for (int e = 0; e < DL; ++e) s_ow[warp][lane * DL + e] = acc.o[e];
   __syncthreads();  // every warp is done reading topj
   // C_i = {0} U sorted Top-k U [lo, i], ascending, for the idx output
-  if (warp == 0) warp_sort_prefix(topj, got, a.kpow2, lane);
+  // (the two-level selection wrote it sorted already)
+  if (warp == 0 && a.kpow2 > 128) warp_sort_prefix(topj, got, a.kpow2, lane);
   if (tid >= 32 && tid < 32 + D) {
     const int dd = tid - 32;
     float M = -INFINITY;

@@ -37,6 +37,8 @@ struct DecodeArgs {
   int cap;              // per-list candidate buffer of the score kernel
   int nstages;          // K staging ring depth of the score kernel
   uint64_t* cand;       // [B, Hq, nchunks, k] chunk-best keys (workspace)
+  int* claims;          // [B, Hkv] unit counters of the tensor-core score
+                        // pass (workspace, zero at launch)
   uint32_t* status;   // device status word (workspace)
   uint64_t wait_ns;   // limit of each pipeline wait (kPipelineWaitNs)
   uint64_t stall_ns;  // failure-path test hook (0: off)

@@ -3,12 +3,16 @@
 // Definition 1 (C_i for the last row), §2.2.3 (Dynamic Top-k), §2.4
 // Corollary 3 (per-query window).
 //
-// Grid (chunks, Hkv, B), about two CTAs per SM; each CTA scores one chunk of
-// the cache of one (batch, kv-head) for the G = Hq/Hkv q-heads reading it:
+// Grid (workers, Hkv, B), about two CTAs per SM; the workers of one (batch,
+// kv-head) share its cache for the G = Hq/Hkv q-heads reading it.  The cache
+// is cut into units of 32 KB (one 128-key tile with both 64-column halves at
+// d = 128, two tiles at d = 64); each worker takes units as it goes (the
+// first ones fixed by its index, the rest claimed from a per-group counter),
+// so that workers which stream faster take more of them, and keeps one
+// candidate list per q-head over the keys it saw.
 //   warp 0     TMA: the group's q rows once (16 rows: the G heads, the rest
-//              of the box ignored), then the chunk's keys in 32 KB copies (one
-//              128-key tile with both 64-column halves at d = 128, two tiles
-//              at d = 64) through a ring of stages.
+//              of the box ignored), then one claimed unit per stage of a ring;
+//              a stage marked empty (position -1) ends the stream.
 //   warp 1     MMA: tcgen05.mma kind::f16 with M = 128 keys and N = 16 heads,
 //              A = the key tile, B = the q rows, fp32 accumulators of 16
 //              columns in TMEM (eight buffers).  The score of key j for head h
@@ -18,7 +22,9 @@
 //              G scores; each goes through the per-head candidate list of the
 //              CUDA-core kernel (the first 512 keys into their own slots, then
 //              admission behind a threshold that only rises, lists cut back to
-//              the head's k by one warp each at every 512 keys).
+//              the head's k by one warp each after every 512 keys).
+// Every list is a union of whole units of the group's keys, so the union of
+// the workers' best-k lists holds the group's global Top-k for each head.
 // The score pass no longer spends CUDA-core instructions on the dot products:
 // the tensor pipe computes them, and the stream is bound by HBM.
 #include "common.cuh"
@@ -57,6 +63,11 @@ struct Shared {
   uint64_t thr[G];
   uint32_t tmem;
   int abort;
+  int spos[kMaxSt];   // first key position of the unit in a stage, -1: end
+  int tpos[kTBufs];   // first key position of the tile in an accumulator
+  int first_tiles;    // tiles of the first stretch that held keys
+  int ended;          // a selector met the end of the stream
+  int stop;           // the selectors leave after this check
   int cnt[G];
   int kk[G];
   int hi[G];
@@ -72,24 +83,38 @@ struct Lay {
   static constexpr size_t k_off = 4096;  // 1024-aligned, after q
 };
 
-// At a check point (all inserts of the stretch done): warp h cuts list h to
-// its head's k keys when it holds more than the limit (that k after the
-// first stretch, else the room the next stretch needs).  Barriers on both
-// sides keep every selector from inserting while a list is being cut.
+// At a check point (all inserts of the stretch done): warp h cuts list h
+// back to its head's k keys, which raises the admission threshold for the
+// next stretch; the keys sit in registers when they fit.  The first check
+// also drops the empty (0) keys of the first stretch's slots, so that later
+// lists hold real keys only.  Barriers on both sides keep every selector
+// from inserting while a list is being cut.  In between, one thread decides
+// for all whether the selectors leave after this check (the stream ended, a
+// wait gave up, or the stretch count reached its bound `last`), so every
+// selector warp takes the same number of barriers.
 template <int G>
 __device__ __forceinline__ void check(uint64_t* buf, int cap, bool first,
-                                      Shared<G>* sh, int sw, int lane) {
+                                      bool last, Shared<G>* sh, int sw,
+                                      int lane) {
   SelBar::sync();
+  if (sw == 0 && lane == 0)
+    sh->stop = (last || sh->ended || *(volatile int*)&sh->abort) ? 1 : 0;
   if (sw < G) {
-    const int n = sh->cnt[sw];
+    const int n = sh->cnt[sw];  // at most kSubKeys on the first check
     const int kk = sh->kk[sw];
-    const int limit = first ? kk : cap - kSubKeys;
-    if (kk > 0 && n > limit && n > kk) {
-      const uint64_t T = warp_cut(buf + (size_t)sw * cap, n, kk, sh->hist[sw],
-                                  lane);
+    if (kk > 0 && (n > kk || (first && n > 0))) {
+      uint64_t* lst = buf + (size_t)sw * cap;
+      uint64_t T;
+      int kept = kk;
+      if (n <= 128) T = warp_cut_regs<4>(lst, n, kk, lane, &kept);
+      else if (n <= 256) T = warp_cut_regs<8>(lst, n, kk, lane, &kept);
+      else if (n <= 512) T = warp_cut_regs<16>(lst, n, kk, lane, &kept);
+      else T = warp_cut(lst, n, kk, sh->hist[sw], lane);  // keys all real
       if (lane == 0) {
-        sh->cnt[sw] = kk;
-        sh->thr[sw] = T;
+        sh->cnt[sw] = kept;
+        // T = 1: the list holds every real key so far, the next stretch
+        // admits any real key
+        sh->thr[sw] = T > 1ull ? T : 0ull;
       }
     }
   }
@@ -130,6 +155,7 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                      int maps3d) {
   using Ly = Lay<D>;
   constexpr int KT = Ly::KT;
+  constexpr int kUnitKeys = KT * kKeys;  // keys per unit (one stage)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -144,14 +170,15 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   // Let the merge kernel (launched as a programmatic dependent) start its
   // independent prologue on SMs this grid releases.
   asm volatile("griddepcontrol.launch_dependents;");
-  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int worker = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int nworkers = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L;
   if (tid == 0) {
     // per q-head of the group: last candidate position and Top-k size
     for (int h = 0; h < G; ++h) {
       const int hq = g * G + h;
-      const bool rep = chunk == 0;
+      const bool rep = worker == 0;
       sh->hi[h] = (L - 1) - row_window(a.W_i, b, a.W_h, hq, a.W, L, a.status,
                                        rep);
       sh->kk[h] = head_k(a.k_h, hq, a.k, a.status, rep);
@@ -165,10 +192,14 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     sm100::mbar_init(&sh->qfull, 1);
     sm100::mbar_init(&sh->never, 1);
     for (int t = 0; t < kTBufs; ++t) {
-      sm100::mbar_init(&sh->tfull[t], 1);
+      // the MMA commit, and the issuer's own arrive after it wrote tpos
+      sm100::mbar_init(&sh->tfull[t], 2);
       sm100::mbar_init(&sh->tempty[t], kSelW / 2);
     }
     sh->abort = 0;
+    sh->first_tiles = 0;
+    sh->ended = 0;
+    sh->stop = 0;
     sm100::fence_barrier_init();
   }
   if (warp == 1) {
@@ -182,36 +213,65 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   int hi = -1;
 #pragma unroll
   for (int h = 0; h < G; ++h) hi = max(hi, sh->hi[h]);
-  // the chunk's candidate keys [c0, c1): positions >= 1, up to the group's
-  // largest last candidate position
-  const int j0 = chunk * a.chunk_len;
-  const int c0 = j0 < 1 ? 1 : j0;
-  const int c1 = (j0 + a.chunk_len < hi + 1) ? j0 + a.chunk_len : hi + 1;
-  const int ntile = c1 > c0 ? (c1 - c0 + kKeys - 1) / kKeys : 0;
-  const int nstage = (ntile + KT - 1) / KT;
+  // the group's candidate keys are positions 1..hi, in units of kUnitKeys
+  // keys from position 0 (position 0 and those past a head's window start
+  // are masked by the selectors)
+  const int nunits = hi >= 1 ? (hi + kUnitKeys) / kUnitKeys : 0;
   volatile int* abort_flag = &sh->abort;
 
   if (warp == 0) {
     // ---------------- TMA producer
-    if (lane == 0 && ntile > 0) {
+    if (lane == 0) {
       sm100::prefetch_tmap(&tmQ);
       sm100::prefetch_tmap(&tmK);
       const int qrow = b * a.Hq + g * G;
-      const int krow = (b * a.Hkv + g) * L + c0;
+      const int krow = (b * a.Hkv + g) * L;
+      int* ctr = a.claims + (size_t)b * a.Hkv + g;
       sm100::mbar_arrive_expect_tx(&sh->qfull, Ly::kQBytes);
       for (int kb = 0; kb < D / 64; ++kb)
         sm100::tma_load_2d(sQ + kb * (kN * 128), &tmQ, &sh->qfull, kb * 64,
                            qrow);
+      // The first NS units of a worker are fixed (worker + i * nworkers);
+      // later ones come from the group's counter, claimed two ahead so that
+      // the atomic's latency hides behind the copies in flight.
+      const int nfixed = NS * nworkers;
+      auto unit_of = [&](int u, int claim) {
+        return u < NS ? worker + u * nworkers : nfixed + claim;
+      };
+      int c_next = 0, c_after = 0;
+      if (nunits > nfixed) {
+        c_next = atomicAdd(ctr, 1);
+        c_after = atomicAdd(ctr, 1);
+      }
       int issued = 0;
-      for (int u = 0; u < nstage; ++u) {
+      // every pass takes a unit no other worker takes (or ends the stream),
+      // so there are at most nunits + 1 passes; the bound only guards that
+      for (int u = 0; u <= nunits + NS; ++u) {
+        int unit = u < NS ? unit_of(u, 0) : unit_of(u, c_next);
+        if (u == nunits + NS) {
+          raise_flag(a.status, kErrInternal);
+          unit = nunits;  // end the stream
+        }
+        if (u >= NS) {
+          c_next = c_after;
+          if (unit < nunits) c_after = atomicAdd(ctr, 1);
+        }
         const int s = u % NS;
         const uint32_t ph = (u / NS) & 1;
         if (u >= NS &&
             !sm100::wait_or_abort(&sh->empty[s], ph ^ 1, abort_flag, a.status,
                                   a.wait_ns))
           break;
+        issued = u + 1;
+        if (unit >= nunits) {
+          // end of the stream: a stage without data
+          sh->spos[s] = -1;
+          sm100::mbar_arrive(&sh->full[s]);
+          break;
+        }
         unsigned char* dst = sK + (size_t)s * kStage;
-        const int row = krow + u * KT * kKeys;
+        const int row = krow + unit * kUnitKeys;
+        sh->spos[s] = unit * kUnitKeys;
         sm100::mbar_arrive_expect_tx(&sh->full[s], kStage);
         if (D == 64) {
           sm100::tma_load_2d(dst, &tmK, &sh->full[s], 0, row);
@@ -222,7 +282,6 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
             sm100::tma_load_2d(dst + kb * 16384, &tmK, &sh->full[s], kb * 64,
                                row);
         }
-        issued = u + 1;
       }
       // every copy this thread started must land before the CTA can exit
       bool drained = sm100::mbar_wait(&sh->qfull, 0, kDrainWaitNs);
@@ -233,11 +292,21 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
-    if (lane == 0 && ntile > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kKeys, kN);
       const uint32_t aq = sm100::smem_u32(sQ);
       const uint32_t ak = sm100::smem_u32(sK);
-      int tt = 0;
+      int tt = 0, real = 0;
+      bool ok = true;
+      // the next accumulator buffer, once the selectors have released it
+      auto take_buf = [&]() -> int {
+        const int tb = tt & (kTBufs - 1);
+        if (tt >= kTBufs &&
+            !sm100::wait_or_abort(&sh->tempty[tb], ((tt / kTBufs) & 1) ^ 1,
+                                  abort_flag, a.status, a.wait_ns))
+          return -1;
+        return tb;
+      };
       if (a.stall_ns) {
         // Failure-path test hook: wait on a barrier that nothing signals, so
         // the wait runs out, raises the time-out flag and aborts every wait
@@ -246,22 +315,36 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       }
       if (sm100::wait_or_abort(&sh->qfull, 0, abort_flag, a.status,
                                a.wait_ns)) {
-        bool ok = true;
-        for (int u = 0; u < nstage && ok; ++u) {
+        for (int u = 0; ok; ++u) {
           const int s = u % NS;
           if (!sm100::wait_or_abort(&sh->full[s], (u / NS) & 1, abort_flag,
                                     a.status, a.wait_ns))
             break;
+          const int pos = *(volatile int*)&sh->spos[s];
+          if (pos < 0) {
+            // end of the stream: two empty tiles, so that both selector
+            // halves (alternate tiles) meet one
+            for (int e = 0; e < 2 && ok; ++e) {
+              const int tb = take_buf();
+              if (tb < 0) {
+                ok = false;
+                break;
+              }
+              sh->tpos[tb] = -1;
+              sm100::mbar_arrive(&sh->tfull[tb]);
+              sm100::mbar_arrive(&sh->tfull[tb]);
+              ++tt;
+            }
+            break;
+          }
 #pragma unroll
           for (int q = 0; q < KT; ++q) {
-            if (tt >= ntile) break;
-            const int tb = tt & (kTBufs - 1);
-            if (tt >= kTBufs &&
-                !sm100::wait_or_abort(&sh->tempty[tb], ((tt / kTBufs) & 1) ^ 1,
-                                      abort_flag, a.status, a.wait_ns)) {
+            const int tb = take_buf();
+            if (tb < 0) {
               ok = false;
               break;
             }
+            sh->tpos[tb] = pos + q * kKeys;
             sm100::tc_fence_after();
             const uint32_t kt = ak + s * kStage + q * 16384;
 #pragma unroll
@@ -273,15 +356,17 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                               kk > 0 ? 1u : 0u);
             }
             sm100::mma_commit(&sh->tfull[tb]);
+            sm100::mbar_arrive(&sh->tfull[tb]);  // releases the tpos write
             ++tt;
+            real = tt;
           }
           sm100::mma_commit(&sh->empty[s]);
         }
       }
       // The last commit covers every MMA issued: wait for it before exit.
-      if (tt > 0 &&
-          !sm100::mbar_wait(&sh->tfull[(tt - 1) & (kTBufs - 1)],
-                            ((tt - 1) / kTBufs) & 1, kDrainWaitNs))
+      if (real > 0 &&
+          !sm100::mbar_wait(&sh->tfull[(real - 1) & (kTBufs - 1)],
+                            ((real - 1) / kTBufs) & 1, kDrainWaitNs))
         raise_flag(a.status, kErrTimeout);
     }
   } else {
@@ -298,10 +383,12 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
     Lse2 ml[G];
     uint64_t thr[G];
     float thr_f[G];
-    const int nstretch = (ntile + kStretchTiles - 1) / kStretchTiles;
-    const int first_keys = min(c1 - c0, kSubKeys);
+    bool done = false;  // this half met the end of the stream
+    // A worker sees at most every unit's tiles and the two end tiles: the
+    // stretch count is bounded by that (a longer run is an internal error).
+    const int max_stretch = (nunits * KT + 2 + kStretchTiles - 1) / kStretchTiles;
 #pragma unroll 1
-    for (int m = 0; m < nstretch; ++m) {
+    for (int m = 0;; ++m) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         thr[h] = sh->thr[h];
@@ -309,13 +396,24 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       }
 #pragma unroll 1
       for (int t = m * kStretchTiles + half;
-           t < min(ntile, (m + 1) * kStretchTiles); t += 2) {
+           t < (m + 1) * kStretchTiles && !done; t += 2) {
         const int tb = t & (kTBufs - 1);
         const bool ok = __all_sync(
             0xFFFFFFFFu,
             sm100::wait_or_abort(&sh->tfull[tb], (t / kTBufs) & 1, abort_flag,
                                  a.status, a.wait_ns));
-        if (!ok) continue;
+        if (!ok) {
+          done = true;
+          break;
+        }
+        const int pos = *(volatile int*)&sh->tpos[tb];
+        if (pos < 0) {
+          done = true;
+          if (lane == 0) sh->ended = 1;
+          break;
+        }
+        if (m == 0 && lane == 0 && (sw & 3) == 0)
+          atomicMax(&sh->first_tiles, t + 1);
         uint32_t v[G];
         sm100::tc_fence_after();
         tmem_ld_g<G>(tl + tb * kN, v);
@@ -323,8 +421,8 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         sm100::tc_fence_before();
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&sh->tempty[tb]);
-        const int j = c0 + t * kKeys + kq;
-        const bool in = j < c1;
+        const int j = pos + kq;
+        const bool in = j >= 1 && j <= hi;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float sc = __uint_as_float(v[h]);
@@ -333,28 +431,33 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
             if (cand) ml[h].add(sc * sl2);
           }
           if (m == 0) {
-            // first stretch: every key goes in, at its own slot (a position
-            // past this head's window start goes in as an empty key)
-            if (in)
-              buf[(size_t)h * cap + (j - c0)] =
-                  cand ? make_key(sc, (uint32_t)j) : 0ull;
+            // first stretch: every key of the tile goes in at its own slot
+            // (a key outside this head's candidates as an empty key)
+            buf[(size_t)h * cap + t * kKeys + kq] =
+                cand ? make_key(sc, (uint32_t)j) : 0ull;
           } else if (cand && sc >= thr_f[h]) {
             const uint64_t key = make_key(sc, (uint32_t)j);
             if (key > thr[h]) {
-              const int pos = atomicAdd(&sh->cnt[h], 1);
-              buf[(size_t)h * cap + pos] = key;
+              const int p = atomicAdd(&sh->cnt[h], 1);
+              buf[(size_t)h * cap + p] = key;
             }
           }
         }
       }
       if (m == 0) {
-        // the first stretch filled slots 0..first_keys-1 of every list
+        // the first stretch filled the slots of its tiles that held keys
+        // (a prefix of the worker's tiles)
         SelBar::sync();
-        if (tid - 64 < G) sh->cnt[tid - 64] = sh->kk[tid - 64] > 0 ? first_keys : 0;
+        if (tid - 64 < G)
+          sh->cnt[tid - 64] = sh->kk[tid - 64] > 0 ? sh->first_tiles * kKeys : 0;
       }
-      check<G>(buf, cap, m == 0, sh, sw, lane);
+      check<G>(buf, cap, m == 0, m >= max_stretch, sh, sw, lane);
+      if (sh->stop) {
+        if (m >= max_stretch && !sh->ended && !*abort_flag && tid == 64)
+          raise_flag(a.status, kErrInternal);
+        break;
+      }
     }
-    check<G>(buf, cap, true, sh, sw, lane);
     if constexpr (MASS) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -372,19 +475,16 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         Lse2 c;
         for (int w = 0; w < kSelW; ++w) c.merge(sh->ml[w][h].x, sh->ml[w][h].y);
         const size_t lst =
-            ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + chunk;
+            ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + worker;
         a.cand_ml[lst] = make_float2(c.m, c.l);
       }
     }
-    // this chunk's best keys per q-head; empty slots get key 0
-#pragma unroll 1
-    for (int h = 0; h < G; ++h) {
+    // this worker's best keys per q-head; empty slots get key 0
+    for (int e = tid - 64; e < G * a.k; e += kSelT) {
+      const int h = e / a.k, r = e - h * a.k;
       const size_t lst =
-          ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + chunk;
-      uint64_t* out = a.cand + lst * a.k;
-      const int cnt = sh->cnt[h];
-      for (int e = tid - 64; e < a.k; e += kSelT)
-        out[e] = e < cnt ? buf[(size_t)h * cap + e] : 0ull;
+          ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + worker;
+      a.cand[lst * a.k + r] = r < sh->cnt[h] ? buf[(size_t)h * cap + r] : 0ull;
     }
   }
   __syncwarp();  // reconverge single-lane roles before the CTA barrier

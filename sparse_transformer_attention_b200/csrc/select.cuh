@@ -183,4 +183,116 @@ __device__ __forceinline__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint3
   return prefix;
 }
 
+// ---------------------------------------------------------------- one warp,
+// keys in registers (element e = t * 32 + lane in v[t]; key 0 marks an
+// absent element and is never counted or kept; the nonzero keys are unique)
+
+// Load n keys from src (shared or global memory) into registers, 0 past n.
+template <int NPL>
+__device__ __forceinline__ void warp_load_keys(const uint64_t* src, int n,
+                                               uint64_t (&v)[NPL], int lane) {
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    const int e = t * 32 + lane;
+    v[t] = e < n ? src[e] : 0ull;
+  }
+}
+
+// The kk-th largest nonzero key (kk >= 1), or 1 when at most kk keys are
+// nonzero: in both cases exactly min(kk, nonzero) keys are >= the result.
+// Bisection on the high words, from the common prefix of the smallest and
+// the largest, then on the low words of the keys whose high word is the
+// chosen one; each count is one warp reduction, and the search stops at the
+// first probe that leaves exactly kk keys above it.
+template <int NPL>
+__device__ __forceinline__ uint64_t warp_kth(const uint64_t (&v)[NPL], int kk) {
+  constexpr unsigned kAll = 0xFFFFFFFFu;
+  uint32_t hw[NPL];
+  uint32_t nz = 0u, mx = 0u, mn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    hw[t] = (uint32_t)(v[t] >> 32);
+    const bool real = v[t] != 0ull;
+    nz += real;
+    mx = real ? max(mx, hw[t]) : mx;
+    mn = real ? min(mn, hw[t]) : mn;
+  }
+  nz = __reduce_add_sync(kAll, nz);
+  if (nz <= (uint32_t)kk) return 1ull;
+  mx = __reduce_max_sync(kAll, mx);
+  mn = __reduce_min_sync(kAll, mn);
+  // Real scores have ord codes of at least 0x007FFFFF in the high word, so
+  // every probe below (>= 1) leaves the absent keys out.
+  const uint32_t diff = mn ^ mx;
+  const int nb = diff ? 32 - __clz(diff) : 0;
+  uint32_t th = nb == 32 ? 0u : (mn >> nb) << nb;
+#pragma unroll 1
+  for (int bit = nb - 1; bit >= 0; --bit) {
+    const uint32_t c = th | (1u << bit);
+    uint32_t m = 0u;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) m += hw[t] >= c;
+    m = __reduce_add_sync(kAll, m);
+    if (m >= (uint32_t)kk) {
+      th = c;
+      if (m == (uint32_t)kk) return (uint64_t)th << 32;
+    }
+  }
+  // th is the kk-th largest high word; fewer than kk keys lie above it
+  uint32_t above = 0u;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) above += hw[t] > th;
+  above = __reduce_add_sync(kAll, above);
+  const uint32_t need = (uint32_t)kk - above;
+  uint32_t tl = 0u;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t c = tl | (1u << bit);
+    uint32_t m = 0u;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t)
+      m += hw[t] == th && (uint32_t)v[t] >= c;
+    m = __reduce_add_sync(kAll, m);
+    if (m >= need) {
+      tl = c;
+      if (m == need) break;
+    }
+  }
+  return ((uint64_t)th << 32) | tl;
+}
+
+// Write the keys >= T (T >= 1) to out[0..), in element order; returns how
+// many.  out may alias the source of v: every lane has its keys in
+// registers before the first ballot.
+template <int NPL>
+__device__ __forceinline__ int warp_keep(const uint64_t (&v)[NPL], uint64_t T,
+                                         uint64_t* out, int lane) {
+  int w = 0;
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    const bool keep = v[t] >= T;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) out[w + __popc(bal & below)] = v[t];
+    w += __popc(bal);
+  }
+  return w;
+}
+
+// One warp cuts lst[0..n) (n <= 32 * NPL, kk >= 1, nonzero keys unique)
+// to its best kk keys in place, dropping the absent (0) keys; returns the
+// kk-th largest key (or 1 when at most kk keys are nonzero, which are then
+// all kept) and sets *kept to the number of keys left.
+template <int NPL>
+__device__ __forceinline__ uint64_t warp_cut_regs(uint64_t* lst, int n, int kk,
+                                                  int lane, int* kept) {
+  uint64_t v[NPL];
+  warp_load_keys<NPL>(lst, n, v, lane);
+  const uint64_t T = warp_kth<NPL>(v, kk);
+  __syncwarp();
+  *kept = warp_keep<NPL>(v, T, lst, lane);
+  __syncwarp();
+  return T;
+}
+
 }  // namespace ca

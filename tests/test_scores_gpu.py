@@ -58,7 +58,9 @@ def test_decode_carried_scores(name):
     assert ca.condensate_attn_status(ws) == ca.CA_OK
     nch = ca.condensate_attn_decode_chunks(w.B, w.n, w.Hkv, w.k)
     per_head = nch * w.k
-    body = ws[256:256 + w.B * w.Hq * per_head * 8].cpu().numpy().view(np.uint64)
+    # after the status area and the [B, Hkv] work counters (256-byte rounded)
+    off = 256 + (w.B * w.Hkv * 4 + 255) // 256 * 256
+    body = ws[off:off + w.B * w.Hq * per_head * 8].cpu().numpy().view(np.uint64)
     G = w.Hq // w.Hkv
     total = 0
     for b in range(w.B):
