@@ -4,23 +4,28 @@
 // Corollary 3 (per-query window), §5.2.2 (select, then attend on the subset).
 //
 // Launch 1, decode_score_topk: grid (chunks, Hkv, B), about two CTAs per SM.
-// One producer thread streams the chunk's contiguous K rows into a ring of
-// 32 KiB shared-memory stages with bulk asynchronous copies (no multicast),
-// so the loads stay deep in flight whatever the compute warps are doing.
-// Eight compute warps read each K row once from shared memory (8 lanes per
-// row, 16-byte reads, conflict-free), score all G = Hq/Hkv q-heads of the
-// group from the same bytes with packed fp32 FMAs, and keep a per-head
-// candidate buffer in shared memory behind a threshold that only rises.
-// Buffers are cut back to exactly the best k keys by a radix select over
-// the compute warps; the chunk's best k keys per q-head go to the workspace.
-// The union of the chunks' best-k lists contains the global Top-k, since
-// every global Top-k member is among the best k of its own chunk.
+// With bf16 inputs the tensor-core pass (decode_tc.cu) runs instead, with
+// the same outputs; this CUDA-core pass serves fp32 inputs.  One producer
+// thread streams the chunk's contiguous K rows into a ring of 32 KiB
+// shared-memory stages with bulk asynchronous copies (no multicast), so the
+// loads stay deep in flight whatever the compute warps are doing.  Eight
+// compute warps read each K row once from shared memory (8 lanes per row,
+// 16-byte reads, conflict-free), score all G = Hq/Hkv q-heads of the group
+// from the same bytes with packed fp32 FMAs, and keep a per-head candidate
+// buffer in shared memory behind a threshold that only rises.  Buffers are
+// cut back to exactly the best k keys by a radix select over the compute
+// warps; the chunk's best k keys per q-head go to the workspace.  The union
+// of the lists contains the global Top-k, since every global Top-k member
+// is among the best k of its own chunk.
 //
 // Launch 2, decode_merge_attend: grid (Hq, B).  Half of each CTA gathers the
-// anchor and window rows and runs their fp32 online softmax while the other
-// half merges the chunk lists into the exact Top-k (radix select), writes
-// C_i in ascending order and accumulates the Top-k rows, whose scores come
-// with their keys; the two partial softmax states are then combined.
+// anchor and window rows into its fp32 online softmax while the score grid
+// drains (they do not depend on the selection); the other half merges the
+// lists into the exact Top-k (for k <= 128: a floor from each list's best
+// few keys, the exact m-th best of the keys at or above it, ranks for
+// ascending positions; else a radix select); then all warps accumulate the
+// Top-k rows, whose scores come with their keys, and the per-warp softmax
+// states are combined.
 #include "common.cuh"
 #include "decode.cuh"
 #include "launch.cuh"
@@ -430,64 +435,49 @@ struct Online {
   }
 };
 
-// Merge, first level: warp gw keeps the best kh of its share of the
-// q-head's ncand worker keys (read from global memory straight into
-// registers) and appends them to lvl at an offset taken from *s_n.
-template <int NPL>
-__device__ __forceinline__ void merge_level1(const uint64_t* src, int n,
-                                             int kh, uint64_t* lvl, int* s_n,
-                                             int lane) {
-  uint64_t v[NPL];
-  warp_load_keys<NPL>(src, n, v, lane);
-  const uint64_t T = warp_kth<NPL>(v, kh);
-  uint32_t cnt = 0u;
+// The r best keys of one worker list lst[0..k) (k <= 128, read by one warp)
+// to out[0..r), largest first, 0 once the list runs out.
+__device__ __forceinline__ void list_top_r(const uint64_t* lst, int k, int r,
+                                           uint64_t* out, int lane) {
+  uint64_t v[4];
 #pragma unroll
-  for (int t = 0; t < NPL; ++t) cnt += v[t] >= T;
-  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-  int base = 0;
-  if (lane == 0 && cnt) base = atomicAdd(s_n, (int)cnt);
-  base = __shfl_sync(0xFFFFFFFFu, base, 0);
-  warp_keep<NPL>(v, T, lvl + base, lane);
+  for (int t = 0; t < 4; ++t) {
+    const int e = t * 32 + lane;
+    v[t] = e < k ? lst[e] : 0ull;
+  }
+#pragma unroll 1
+  for (int q = 0; q < r; ++q) {
+    const uint64_t mx = warp_max_u64(max(max(v[0], v[1]), max(v[2], v[3])));
+    if (lane == 0) out[q] = mx;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) v[t] = v[t] == mx ? 0ull : v[t];
+  }
 }
 
-// Merge, second level (one warp): the best m (1 <= m <= 128) of the n
-// first-level keys in lvl, written as (position, score) pairs in ascending
-// position order to topj/tops[0..); returns how many were selected.  lvl is
-// reused as scratch.
+// One warp: the m-th largest of the leading r keys of each list in src
+// (list c starts at src[c * k]; n = lists * r <= 32 * NPL), or 1 when at
+// most m of them are nonzero.
 template <int NPL>
-__device__ __forceinline__ int merge_level2(uint64_t* lvl, int n, int m,
-                                            uint32_t* topj, float* tops,
-                                            int lane) {
+__device__ __forceinline__ uint64_t warp_kth_lead(const uint64_t* src, int k,
+                                                  int r, int n, int m,
+                                                  int lane) {
   uint64_t v[NPL];
-  warp_load_keys<NPL>(lvl, n, v, lane);
-  const uint64_t T = warp_kth<NPL>(v, m);
-  // the selected keys as (position << 32 | score bits), packed to lvl[0..)
 #pragma unroll
-  for (int t = 0; t < NPL; ++t)
-    if (v[t] >= T)
-      v[t] = ((uint64_t)key_index(v[t]) << 32) |
-             __float_as_uint(key_score(v[t]));
-    else
-      v[t] = 0ull;
-  __syncwarp();
-  const int got = warp_keep<NPL>(v, 1ull, lvl, lane);
-  __syncwarp();
-  uint64_t srt[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
+  for (int t = 0; t < NPL; ++t) {
     const int e = t * 32 + lane;
-    srt[t] = e < got && e < 128 ? lvl[e] : ~0ull;
+    v[t] = e < n ? src[(size_t)(e / r) * k + e % r] : 0ull;
   }
-  warp_bitonic64<4>(srt, lane);
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int e = t * 32 + lane;
-    if (e < got && e < 128) {
-      topj[e] = (uint32_t)(srt[t] >> 32);
-      tops[e] = __uint_as_float((uint32_t)srt[t]);
-    }
-  }
-  return got;
+  return warp_kth<NPL>(v, m);
+}
+
+// One warp: the m-th largest of the n keys in src (n <= 32 * NPL), or 1
+// when at most m are nonzero.
+template <int NPL>
+__device__ __forceinline__ uint64_t warp_kth_of(const uint64_t* src, int n,
+                                                int m, int lane) {
+  uint64_t v[NPL];
+  warp_load_keys<NPL>(src, n, v, lane);
+  return warp_kth<NPL>(v, m);
 }
 
 template <typename T, int D, typename TO>
@@ -500,7 +490,9 @@ decode_merge_attend(DecodeArgs a) {
   const int k = a.k;
   const int ncand = a.nchunks * k;
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem);           // [ncand]
-  uint32_t* topj = reinterpret_cast<uint32_t*>(cand + ncand);   // [kpow2]
+  uint64_t* surv = cand + ncand;                                // [ncand]
+  uint64_t* pairs = surv + ncand;                               // [128]
+  uint32_t* topj = reinterpret_cast<uint32_t*>(pairs + 128);    // [kpow2]
   float* tops = reinterpret_cast<float*>(topj + a.kpow2);       // [kpow2]
   SelectState<1>* st = reinterpret_cast<SelectState<1>*>(tops + a.kpow2);
   __shared__ int s_n, s_kk, s_m;
@@ -508,6 +500,7 @@ decode_merge_attend(DecodeArgs a) {
   __shared__ float s_mw[NW], s_lw[NW];
   __shared__ float s_ow[NW][D];
   __shared__ float s_wm[8], s_wl[8], s_s0;  // window+anchor states; anchor score
+  __shared__ int s_seg[8];                     // survivors per merge warp
 
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -533,9 +526,26 @@ decode_merge_attend(DecodeArgs a) {
                 ((size_t)b * a.Hkv + g) * (size_t)L * D + lane * DL;
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e)/sqrt(d)
   Online<DL> acc;
+  {
+    // ask L2 for the anchor and (the first 512) window rows of K and V at
+    // once, so that the window gathers below wait for one L2 round trip
+    // rather than one HBM round trip per batch of rows
+    constexpr int kLines = D * (int)sizeof(T) / 128;
+    const int64_t nwin = min(anc + (i - lo + 1), (int64_t)512);
+    const char* kb = reinterpret_cast<const char*>(Kg - lane * DL);
+    const char* vb = reinterpret_cast<const char*>(Vg - lane * DL);
+    for (int64_t e = tid; e < nwin * kLines; e += kMergeThreads) {
+      const int64_t row = e / kLines, ln = e % kLines;
+      const int64_t j = (anc && row == 0) ? 0 : lo + (row - anc);
+      const size_t o = (size_t)j * D * sizeof(T) + (size_t)ln * 128;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(kb + o));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(vb + o));
+    }
+  }
 
   if (warp >= 8) {
-    // ---------------- anchor and window rows (no dependence on selection)
+    // ---------------- anchor and window rows (no dependence on selection;
+    // they run while the score grid drains)
     const int64_t nwin = anc + (i - lo + 1);
 #pragma unroll 1
     for (int64_t e0 = gw; e0 < nwin; e0 += 8 * UG) {
@@ -580,63 +590,154 @@ decode_merge_attend(DecodeArgs a) {
       }
     }
   } else {
-    // ---------------- merge the chunk lists into the exact Top-k
+    // ---------------- merge the worker lists into the exact Top-k
     // The lists are written by the score kernel, which may still be
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
-    if (a.kpow2 <= 128) {
-      // Two levels of register-resident selection: each warp keeps the best
-      // m of an eighth of the keys, then warp 0 the best m of those (at most
-      // 8 m <= 1024 keys), written in ascending position order.
-      if (gtid == 0) {
-        s_n = 0;
-        s_m = 0;
+    // every list into shared memory at once: 16-byte asynchronous copies
+    // (the list area of a head starts 16-byte aligned: k keys per list,
+    // 8 bytes each, and the workspace lists start at a 256-byte boundary;
+    // an odd k leaves the head's area 8-byte aligned: then plain loads)
+    const bool async_ok = (((uintptr_t)src) & 15u) == 0;
+    if (async_ok) {
+      for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         (uint32_t)__cvta_generic_to_shared(cand + e)),
+                     "l"(src + e)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
+    } else {
+      for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
+    }
+    // k <= 128: a floor first.  With each list's r = ceil(m / lists) best
+    // keys, the m-th largest of those, F, has m keys at or above it, so the
+    // global m-th best key is >= F and only keys >= F can be selected
+    // (about m survive).  The tensor-core pass writes those r keys at the
+    // front of each list: then warp 0 reads them from global memory while
+    // the copies land.
+    const bool fast = a.kpow2 <= 128;
+    const int r = m > 0 ? (m + a.nchunks - 1) / a.nchunks : 0;
+    const int nt = a.nchunks * r;
+    const bool use_floor = fast && m > 0 && r <= kDecodeTopR && nt <= 512;
+    const bool lead = use_floor && a.top_first;
+    if (lead && gw == 0) {
+      const uint64_t F = nt <= 128 ? warp_kth_lead<4>(src, k, r, nt, m, lane)
+                                   : warp_kth_lead<16>(src, k, r, nt, m, lane);
+      if (lane == 0) s_T = F;
+    }
+    if (async_ok) asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (gtid == 0) {
+      s_n = 0;
+      s_m = 0;
+      s_kk = m > 0 ? m : 1;
+      if (!lead) s_T = fast ? 1ull : 0ull;  // 1: no floor, real keys only
+    }
+    MergeBar::sync();
+    if (fast) {
+      // Loops stay rolled: this code runs once per CTA, from a cold
+      // instruction cache.
+      if (use_floor && !lead) {
+        for (int c = gw; c < a.nchunks; c += 8)
+          list_top_r(cand + (size_t)c * k, k, r, surv + (size_t)c * r, lane);
+        MergeBar::sync();
+        if (gw == 0) {
+          const uint64_t F = nt <= 128 ? warp_kth_of<4>(surv, nt, m, lane)
+                                       : warp_kth_of<16>(surv, nt, m, lane);
+          if (lane == 0) s_T = F;
+        }
+        MergeBar::sync();
+      }
+      const uint64_t F = s_T;
+      // survivors (keys >= F): warp gw packs those of its slice to the same
+      // slice of surv, and asks L2 for their V rows, which the Top-k
+      // accumulation reads next
+      const int per = (ncand + 7) / 8;
+      if (m > 0) {
+        const int beg = min(ncand, gw * per), end = min(ncand, beg + per);
+        int w = 0;
+        for (int e0 = beg; e0 < end; e0 += 32) {
+          const int e = e0 + lane;
+          const uint64_t key = e < end ? cand[e] : 0ull;
+          const bool keep = key >= F;  // F >= 1: real keys only
+          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+          if (keep) {
+            surv[beg + w + __popc(bal & ((1u << lane) - 1u))] = key;
+            const char* row = reinterpret_cast<const char*>(
+                Vg - lane * DL + (size_t)key_index(key) * D);
+            for (int o = 0; o < D * (int)sizeof(T); o += 128)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(row + o));
+          }
+          w += __popc(bal);
+        }
+        if (lane == 0) s_seg[gw] = w;
       }
       MergeBar::sync();
       if (m > 0) {
-        const int per = (ncand + 7) / 8;
-        const int beg = min(ncand, gw * per);
-        const int cnt = min(ncand - beg, per);
-        if (per <= 128) merge_level1<4>(src + beg, cnt, m, cand, &s_n, lane);
-        else if (per <= 256) merge_level1<8>(src + beg, cnt, m, cand, &s_n, lane);
-        else if (per <= 512) merge_level1<16>(src + beg, cnt, m, cand, &s_n, lane);
-        else merge_level1<32>(src + beg, cnt, m, cand, &s_n, lane);
+        int off[8], ns = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          off[c] = ns;
+          ns += s_seg[c];
+        }
+        // survivors, contiguous, into cand (no longer read)
+        auto gather = [&](int e) -> uint64_t {
+          int c = 0;
+#pragma unroll
+          for (int q = 1; q < 8; ++q) c = e >= off[q] ? q : c;
+          return surv[(size_t)c * per + (e - off[c])];
+        };
+        if (ns <= 512) {
+          if (gw == 0) {
+            for (int e = lane; e < ns; e += 32) cand[e] = gather(e);
+            __syncwarp();
+            const uint64_t Tm = ns <= 128 ? warp_kth_of<4>(cand, ns, m, lane)
+                                          : warp_kth_of<16>(cand, ns, m, lane);
+            int got = 0;
+            for (int e0 = 0; e0 < ns; e0 += 32) {
+              const int e = e0 + lane;
+              const uint64_t key = e < ns ? cand[e] : 0ull;
+              const bool keep = key >= Tm;
+              const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+              const int p = got + __popc(bal & ((1u << lane) - 1u));
+              if (keep && p < 128)
+                pairs[p] = ((uint64_t)key_index(key) << 32) |
+                           __float_as_uint(key_score(key));
+              got += __popc(bal);
+            }
+            if (lane == 0) s_m = got;
+          }
+        } else {
+          // many survivors: radix select over the eight warps
+          for (int e = gtid; e < ns; e += 256) cand[e] = gather(e);
+          if (gtid == 0) s_n = ns;
+          MergeBar::sync();
+          cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T,
+                                                  st, gtid);
+          for (int e = gtid; e < ns; e += 256) {
+            const uint64_t key = cand[e];
+            if (key >= s_T && key != 0ull) {
+              const int p = atomicAdd(&s_m, 1);
+              if (p < 128)
+                pairs[p] = ((uint64_t)key_index(key) << 32) |
+                           __float_as_uint(key_score(key));
+            }
+          }
+        }
       }
       MergeBar::sync();
-      if (m > 0 && gw == 0) {
-        const int n = s_n;
-        int got;
-        if (n <= 128) got = merge_level2<4>(cand, n, m, topj, tops, lane);
-        else if (n <= 256) got = merge_level2<8>(cand, n, m, topj, tops, lane);
-        else if (n <= 512) got = merge_level2<16>(cand, n, m, topj, tops, lane);
-        else got = merge_level2<32>(cand, n, m, topj, tops, lane);
-        if (lane == 0) s_m = got;
+      // ascending positions: each selected key goes to its rank
+      const int got = min(min(s_m, m), 128);
+      if (gtid < got) {
+        const uint64_t my = pairs[gtid];
+        int rank = 0;
+        for (int e = 0; e < got; ++e) rank += pairs[e] < my;
+        topj[rank] = (uint32_t)(my >> 32);
+        tops[rank] = __uint_as_float((uint32_t)my);
       }
     } else {
-      // every list into shared memory at once: 16-byte asynchronous copies
-      // (the list area of a head starts 16-byte aligned: k keys per chunk,
-      // 8 bytes each, and the workspace lists start at a 256-byte boundary;
-      // an odd k leaves the head's area 8-byte aligned: then plain loads)
-      if ((((uintptr_t)src) & 15u) == 0) {
-        for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                           (uint32_t)__cvta_generic_to_shared(cand + e)),
-                       "l"(src + e)
-                       : "memory");
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      } else {
-        for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
-      }
-      if (gtid == 0) {
-        s_n = 0;
-        s_m = 0;
-        s_kk = m > 0 ? m : 1;
-      }
-      MergeBar::sync();
       // Every chunk list holds its chunk's best k keys, so the largest of the
       // lists' smallest keys, T0, is at most the global k-th best key (the
       // chunk that has it alone holds k keys >= T0): only keys >= T0 can be
@@ -793,6 +894,7 @@ void score_smem(int k, int* cap, int* nstages, size_t* bytes) {
 
 template <typename T, int D, int G>
 cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
+  a.top_first = 0;
   size_t smem1;
   score_smem<T, D, G>(a.k, &a.cap, &a.nstages, &smem1);
   cudaError_t e = cudaSuccess;
@@ -807,6 +909,7 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
       if (e != cudaErrorNotSupported) {
         if (e != cudaSuccess) return e;
         done = true;
+        a.top_first = 1;
       }
     }
     if (!done) {
@@ -823,8 +926,8 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
       if (e != cudaSuccess) return e;
     }
   }
-  const size_t smem2 = (size_t)a.nchunks * a.k * 8 + (size_t)a.kpow2 * 8 +
-                       sizeof(SelectState<1>);
+  const size_t smem2 = (size_t)a.nchunks * a.k * 16 + 128 * 8 +
+                       (size_t)a.kpow2 * 8 + sizeof(SelectState<1>);
   dim3 grid2(a.Hq, a.B);
   auto k2 = a.o_bf16 ? decode_merge_attend<T, D, __nv_bfloat16>
                      : decode_merge_attend<T, D, float>;

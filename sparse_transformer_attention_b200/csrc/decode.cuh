@@ -15,6 +15,9 @@ constexpr int kDecodeMaxK = 1024;
 // Upper bound on merged candidates per q-head (chunks x k), so the merge
 // fits in shared memory.
 constexpr int kDecodeMaxMerge = 8192;
+// With k <= 128, each worker list of the tensor-core score pass starts with
+// its r = ceil(m / workers) best keys when r is at most this.
+constexpr int kDecodeTopR = 8;
 
 struct DecodeArgs {
   const void* q;
@@ -34,6 +37,8 @@ struct DecodeArgs {
   int32_t* idx_count;
   int C_max;
   int chunk_len, nchunks, kpow2;
+  int top_first;        // 1: each list starts with its r best keys (see
+                        // kDecodeTopR), written by the tensor-core pass
   int cap;              // per-list candidate buffer of the score kernel
   int nstages;          // K staging ring depth of the score kernel
   uint64_t* cand;       // [B, Hq, nchunks, k] chunk-best keys (workspace)

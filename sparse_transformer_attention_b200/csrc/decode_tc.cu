@@ -232,17 +232,15 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         sm100::tma_load_2d(sQ + kb * (kN * 128), &tmQ, &sh->qfull, kb * 64,
                            qrow);
       // The first NS units of a worker are fixed (worker + i * nworkers);
-      // later ones come from the group's counter, claimed two ahead so that
-      // the atomic's latency hides behind the copies in flight.
+      // later ones come from the group's counter, each claimed one stage
+      // ahead so that the atomic's latency hides behind the copies in
+      // flight (claiming further ahead leaves more work committed to a
+      // worker when the counter runs out).
       const int nfixed = NS * nworkers;
       auto unit_of = [&](int u, int claim) {
         return u < NS ? worker + u * nworkers : nfixed + claim;
       };
-      int c_next = 0, c_after = 0;
-      if (nunits > nfixed) {
-        c_next = atomicAdd(ctr, 1);
-        c_after = atomicAdd(ctr, 1);
-      }
+      int c_next = nunits > nfixed ? atomicAdd(ctr, 1) : 0;
       int issued = 0;
       // every pass takes a unit no other worker takes (or ends the stream),
       // so there are at most nunits + 1 passes; the bound only guards that
@@ -252,10 +250,7 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
           raise_flag(a.status, kErrInternal);
           unit = nunits;  // end the stream
         }
-        if (u >= NS) {
-          c_next = c_after;
-          if (unit < nunits) c_after = atomicAdd(ctr, 1);
-        }
+        if (u >= NS && unit < nunits) c_next = atomicAdd(ctr, 1);
         const int s = u % NS;
         const uint32_t ph = (u / NS) & 1;
         if (u >= NS &&
@@ -479,12 +474,54 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         a.cand_ml[lst] = make_float2(c.m, c.l);
       }
     }
-    // this worker's best keys per q-head; empty slots get key 0
-    for (int e = tid - 64; e < G * a.k; e += kSelT) {
-      const int h = e / a.k, r = e - h * a.k;
-      const size_t lst =
-          ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + worker;
-      a.cand[lst * a.k + r] = r < sh->cnt[h] ? buf[(size_t)h * cap + r] : 0ull;
+    // this worker's best keys per q-head; empty slots get key 0.  With
+    // k <= 128 a list starts with its r best keys, largest first, for the
+    // head's m = min(k_h, candidate positions) and r = ceil(m / workers):
+    // the merge takes a floor from those when r <= kDecodeTopR.
+    if (a.k <= 128) {
+      if (sw < G) {
+        const int h = sw;
+        uint64_t* out =
+            a.cand + (((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks +
+                      worker) * a.k;
+        const int cnt = sh->cnt[h];
+        const int mh = min(sh->kk[h], max(hi_h[h], 0));
+        const int r = mh > 0 ? (mh + nworkers - 1) / nworkers : 0;
+        uint64_t v[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int e = t * 32 + lane;
+          v[t] = e < cnt ? buf[(size_t)h * cap + e] : 0ull;
+        }
+        int w = 0;
+        if (r <= kDecodeTopR) {
+#pragma unroll 1
+          for (; w < r; ++w) {
+            const uint64_t mx =
+                warp_max_u64(max(max(v[0], v[1]), max(v[2], v[3])));
+            if (lane == 0) out[w] = mx;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) v[t] = v[t] == mx ? 0ull : v[t];
+          }
+        }
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const bool keep = v[t] != 0ull;
+          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+          if (keep) out[w + __popc(bal & below)] = v[t];
+          w += __popc(bal);
+        }
+        for (int e = w + lane; e < a.k; e += 32) out[e] = 0ull;
+      }
+    } else {
+      for (int e = tid - 64; e < G * a.k; e += kSelT) {
+        const int h = e / a.k, r = e - h * a.k;
+        const size_t lst =
+            ((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks + worker;
+        a.cand[lst * a.k + r] =
+            r < sh->cnt[h] ? buf[(size_t)h * cap + r] : 0ull;
+      }
     }
   }
   __syncwarp();  // reconverge single-lane roles before the CTA barrier

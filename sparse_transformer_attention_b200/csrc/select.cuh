@@ -187,6 +187,14 @@ __device__ __forceinline__ uint64_t warp_cut(uint64_t* lst, int n, int kk, uint3
 // keys in registers (element e = t * 32 + lane in v[t]; key 0 marks an
 // absent element and is never counted or kept; the nonzero keys are unique)
 
+// Largest of the 64-bit values held by a warp (every lane gets it).
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+  return v;
+}
+
 // Load n keys from src (shared or global memory) into registers, 0 past n.
 template <int NPL>
 __device__ __forceinline__ void warp_load_keys(const uint64_t* src, int n,
