@@ -114,18 +114,29 @@ def job_rate(units_per_rank, world, ms):
     return units_per_rank * world / (ms * 1e-3)
 
 
-def kernel_source_hash():
+# The source files a kernel's code comes from (with every shared header).
+KERNEL_SOURCES = {
+    "decode_score_topk": ("decode_tc.cu", "decode.cu"),
+    "decode_merge_attend": ("decode.cu",),
+    "prefill_score_topk_tc": ("prefill_tc.cu",),
+    "prefill_gather": ("prefill.cu",),
+}
+
+
+def kernel_source_hash(kernel):
     csrc = os.path.join(ROOT, "sparse_transformer_attention_b200", "csrc")
+    own = KERNEL_SOURCES.get(kernel)
     h = hashlib.sha256()
     for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
+        if fn.endswith(".cuh") or (fn.endswith(".cu") and
+                                   (own is None or fn in own)):
             h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel, workload):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources; else None."""
+    the current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -134,7 +145,7 @@ def traffic_for(kernel, workload):
     except ValueError:
         return None
     e = t.get(f"{kernel}/{workload}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
