@@ -204,6 +204,60 @@ CA_API ca_status condensate_attn_decode_ex(
     void* stream);
 
 /*
+ * Sequence-sharded decode: the cache of one sequence (length L, query at
+ * position L-1) split along L over P ranks, rank p holding the contiguous
+ * rows [pos0, pos0 + L_shard) as its own K and V of shape
+ * [B, Hkv, L_shard, d].  The set C_i and the output are those of
+ * condensate_attn_decode on the whole cache (§2.1 Definition 1 for the
+ * last row, §2.2.3 Top-k, §5.2.2 select then attend); the split and the two
+ * exchanges are this library's, not the paper's.  Per rank, in order:
+ *   1. condensate_attn_decode_shard_select: the best min(k, candidates in
+ *      the shard) selection keys of the shard per (batch, q-head), to
+ *      keys_out [B, Hq, k] (64-bit keys as described for
+ *      condensate_attn_decode_chunks, positions in the sequence; best first
+ *      when k <= 128; 0 after them).  bf16 only (the tensor-core score
+ *      pass); CA_ERR_UNSUPPORTED otherwise.
+ *   2. the caller gathers every rank's keys_out into keys_all [P, B, Hq, k]
+ *      in rank order (an all-gather);
+ *   3. condensate_attn_decode_shard_attend: the exact Top-k of the sequence
+ *      from keys_all (the same on every rank), idx / idx_count as
+ *      condensate_attn_decode writes them, and this shard's softmax state
+ *      over its members of C_i to partial [B, Hq, d + 2] fp32: the running
+ *      maximum (log2 domain, scores scaled by log2(e)/sqrt(d)), the sum of
+ *      2^(s - max), then the d sums of 2^(s - max) v (max = -inf and sum 0
+ *      when no member lies in the shard);
+ *   4. the caller gathers every rank's partial into partials [P, B, Hq,
+ *      d + 2] (an all-gather);
+ *   5. condensate_attn_decode_shard_combine: O [B, Hq, d] in o_dtype.
+ * W_i may be NULL; per-head windows, mass and lse outputs are not offered
+ * here.  Workspace: condensate_attn_decode_shard_workspace_size for step 1,
+ * 256 bytes for step 3 (each call clears what it uses).  Pointers are
+ * device pointers, 16-byte aligned (W_i 4-byte); the caller owns every
+ * buffer; errors as for condensate_attn_decode, with pos0 < 0, L_shard < 1
+ * or pos0 + L_shard > L an invalid argument and P * k > 8192 unsupported.
+ */
+CA_API size_t condensate_attn_decode_shard_workspace_size(ca_dtype dtype,
+                                                          int B, int L_shard,
+                                                          int Hq, int Hkv,
+                                                          int d, int k);
+CA_API ca_status condensate_attn_decode_shard_select(
+    const void* q, const void* K, ca_dtype dtype, int B, int L_shard,
+    int pos0, int L, int Hq, int Hkv, int d, int W, int k,
+    const int32_t* W_i, uint64_t* keys_out, void* workspace,
+    size_t workspace_bytes, void* stream);
+CA_API ca_status condensate_attn_decode_shard_attend(
+    const void* q, const void* K, const void* V, ca_dtype dtype, int B,
+    int L_shard, int pos0, int L, int Hq, int Hkv, int d, int W, int k,
+    const int32_t* W_i, const uint64_t* keys_all, int P, float* partial,
+    int32_t* idx, int32_t* idx_count, int C_max, void* workspace,
+    size_t workspace_bytes, void* stream);
+CA_API ca_status condensate_attn_decode_shard_combine(const float* partials,
+                                                      int P, int B, int Hq,
+                                                      int d, void* O,
+                                                      ca_dtype o_dtype,
+                                                      void* stream);
+
+/*
  * Decode without a workspace argument, for callers that cannot allocate
  * device memory or pass a scratch pointer (a plugin whose host exposes no
  * allocator, a fully pre-budgeted memory plan, a fixed interface with no

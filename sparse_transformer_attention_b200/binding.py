@@ -62,6 +62,16 @@ SIGNATURES = {
         (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P,
               _I, _P]),
     "condensate_attn_decode_noalloc_status": (_I, [_P]),
+    "condensate_attn_decode_shard_workspace_size":
+        (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "condensate_attn_decode_shard_select":
+        (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+              ctypes.c_size_t, _P]),
+    "condensate_attn_decode_shard_attend":
+        (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I,
+              _P, _P, _P, _I, _P, ctypes.c_size_t, _P]),
+    "condensate_attn_decode_shard_combine":
+        (_I, [_P, _I, _I, _I, _I, _P, _I, _P]),
     "condensate_attn_status": (_I, [_P, _P]),
     "condensate_attn_test_stall": (_I, [ctypes.c_ulonglong]),
     "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
@@ -269,6 +279,94 @@ def condensate_attn_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         workspace.numel(), _stream(stream))
     _check(code, "condensate_attn_decode_ex")
     return O, idx, idx_count
+
+
+def condensate_attn_decode_shard_workspace_size(dtype: torch.dtype, B: int,
+                                                L_shard: int, Hq: int,
+                                                Hkv: int, d: int,
+                                                k: int) -> int:
+    return int(load().condensate_attn_decode_shard_workspace_size(
+        _dt(dtype), B, L_shard, Hq, Hkv, d, k))
+
+
+def condensate_attn_decode_shard_select(q: torch.Tensor, K: torch.Tensor,
+                                        pos0: int, L: int, W: int, k: int,
+                                        W_i: Optional[torch.Tensor] = None,
+                                        keys_out: Optional[torch.Tensor] = None,
+                                        workspace: Optional[torch.Tensor] = None,
+                                        stream=None) -> torch.Tensor:
+    """Step 1 of the sequence-sharded decode (see the header): this shard's
+    best keys, [B, Hq, k] int64 (the 64-bit keys' bits)."""
+    B, Hq, d = q.shape
+    Hkv, Ls = K.shape[1], K.shape[2]
+    for t, nm in ((q, "q"), (K, "K")):
+        _require(t, nm)
+    if keys_out is None:
+        keys_out = torch.empty((B, Hq, k), dtype=torch.int64, device=q.device)
+    if workspace is None:
+        ws = condensate_attn_decode_shard_workspace_size(q.dtype, B, Ls, Hq,
+                                                         Hkv, d, k)
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    code = load().condensate_attn_decode_shard_select(
+        _ptr(q), _ptr(K), _dt(q.dtype), B, Ls, int(pos0), int(L), Hq, Hkv, d,
+        int(W), int(k), _ptr(W_i), _ptr(keys_out), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_decode_shard_select")
+    return keys_out
+
+
+def condensate_attn_decode_shard_attend(q: torch.Tensor, K: torch.Tensor,
+                                        V: torch.Tensor, pos0: int, L: int,
+                                        W: int, k: int,
+                                        keys_all: torch.Tensor,
+                                        W_i: Optional[torch.Tensor] = None,
+                                        partial: Optional[torch.Tensor] = None,
+                                        idx: Optional[torch.Tensor] = None,
+                                        idx_count: Optional[torch.Tensor] = None,
+                                        C_max: Optional[int] = None,
+                                        workspace: Optional[torch.Tensor] = None,
+                                        stream=None):
+    """Step 3: from every shard's keys keys_all [P, B, Hq, k], this shard's
+    softmax state partial [B, Hq, d + 2] and the sequence's idx/idx_count."""
+    B, Hq, d = q.shape
+    Hkv, Ls = K.shape[1], K.shape[2]
+    P = keys_all.shape[0]
+    for t, nm in ((q, "q"), (K, "K"), (V, "V"), (keys_all, "keys_all")):
+        _require(t, nm)
+    dev = q.device
+    if C_max is None:
+        C_max = min(L, 1 + (int(W_i.max()) if W_i is not None else W) + k)
+    if partial is None:
+        partial = torch.empty((B, Hq, d + 2), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Hq, C_max), dtype=torch.int32, device=dev)
+    if idx_count is None:
+        idx_count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
+    code = load().condensate_attn_decode_shard_attend(
+        _ptr(q), _ptr(K), _ptr(V), _dt(q.dtype), B, Ls, int(pos0), int(L), Hq,
+        Hkv, d, int(W), int(k), _ptr(W_i), _ptr(keys_all), P, _ptr(partial),
+        _ptr(idx), _ptr(idx_count), int(C_max), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(code, "condensate_attn_decode_shard_attend")
+    return partial, idx, idx_count
+
+
+def condensate_attn_decode_shard_combine(partials: torch.Tensor,
+                                         O: Optional[torch.Tensor] = None,
+                                         o_dtype: torch.dtype = torch.float32,
+                                         stream=None) -> torch.Tensor:
+    """Step 5: O [B, Hq, d] from every shard's partials [P, B, Hq, d + 2]."""
+    _require(partials, "partials")
+    P, B, Hq, d2 = partials.shape
+    d = d2 - 2
+    if O is None:
+        O = torch.empty((B, Hq, d), dtype=o_dtype, device=partials.device)
+    code = load().condensate_attn_decode_shard_combine(
+        _ptr(partials), P, B, Hq, d, _ptr(O), _dt(O.dtype), _stream(stream))
+    _check(code, "condensate_attn_decode_shard_combine")
+    return O
 
 
 def condensate_attn_decode_chunks(B: int, L: int, Hkv: int, k: int) -> int:

@@ -92,11 +92,55 @@ ca_status check_common(const void* q, const void* K, const void* V,
   return CA_OK;
 }
 
+
+// Checks shared by the two per-shard steps.
+ca_status check_shard(const void* q, const void* K, ca_dtype dtype, int B,
+                      int L_shard, int pos0, int L, int Hq, int Hkv, int d,
+                      int W, int k, const int32_t* W_i, void* ws) {
+  if (!q || !K) return CA_ERR_INVALID_ARG;
+  if (B < 1 || L_shard < 1 || pos0 < 0 || L < 1 ||
+      (long long)pos0 + L_shard > L || k < 0 || (!W_i && W < 1))
+    return CA_ERR_INVALID_ARG;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return CA_ERR_INVALID_ARG;
+  if (dtype != CA_F32 && dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return CA_ERR_UNSUPPORTED;
+  if (!group_ok(Hq, Hkv)) return CA_ERR_UNSUPPORTED;
+  if (k > ca::kDecodeMaxK) return CA_ERR_UNSUPPORTED;
+  if (!ws) return CA_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(ws) ||
+      (W_i && ((uintptr_t)W_i & 3u)))
+    return CA_ERR_ALIGNMENT;
+  return CA_OK;
+}
+
+void shard_args(ca::DecodeArgs& a, const void* q, const void* K,
+                const void* V, int B, int L_shard, int pos0, int L, int Hq,
+                int Hkv, int W, int k, const int32_t* W_i, void* ws) {
+  a.q = q; a.K = K; a.V = V;
+  a.B = B; a.L = L_shard; a.Hq = Hq; a.Hkv = Hkv; a.W = W; a.k = k;
+  a.Lg = L; a.pos0 = pos0;
+  a.W_i = W_i; a.W_h = nullptr; a.k_h = nullptr;
+  a.mass = nullptr; a.lse = nullptr; a.cand_ml = nullptr;
+  a.O = nullptr; a.o_bf16 = 0;
+  a.idx = nullptr; a.idx_count = nullptr; a.C_max = 0;
+  a.keys_out = nullptr; a.partial = nullptr;
+  a.kpow2 = next_pow2(k > 1 ? k : 2);
+  a.status = (uint32_t*)ws;
+  a.claims = (int*)((char*)ws + ca::kStatusBytes);
+  a.wait_ns = ca::kPipelineWaitNs;
+  a.stall_ns = g_stall_ns.load();
+}
+
+ca_status launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return CA_OK;
+  return e == cudaErrorNotSupported ? CA_ERR_UNSUPPORTED : CA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
 
-int condensate_attn_version(void) { return 200; }
+int condensate_attn_version(void) { return 300; }
 
 const char* condensate_attn_status_string(ca_status s) {
   switch (s) {
@@ -168,10 +212,103 @@ ca_status condensate_attn_decode_ex(const void* q, const void* K,
   a.cand = (uint64_t*)((char*)workspace + cleared);
   a.cand_ml = (float2*)((char*)a.cand +
                         decode_lists_bytes(B, Hq, a.nchunks, k));
+  a.Lg = L;
+  a.pos0 = 0;
+  a.mode = ca::kDecodeAttend;
+  a.keys_out = nullptr;
+  a.partial = nullptr;
   a.wait_ns = ca::kPipelineWaitNs;
   a.stall_ns = g_stall_ns.load();
   cudaError_t e = ca::decode_launch(a, dtype == CA_BF16, d, s);
   return e == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+}
+
+// ------------------------------------------------- sequence-sharded decode
+
+size_t condensate_attn_decode_shard_workspace_size(ca_dtype dtype, int B,
+                                                   int L_shard, int Hq,
+                                                   int Hkv, int d, int k) {
+  if (!sizes_ok(dtype, B, 1, L_shard, Hq, Hkv, d, 1, k)) return 0;
+  return decode_ws(B, L_shard, Hq, Hkv, k);
+}
+
+ca_status condensate_attn_decode_shard_select(
+    const void* q, const void* K, ca_dtype dtype, int B, int L_shard,
+    int pos0, int L, int Hq, int Hkv, int d, int W, int k,
+    const int32_t* W_i, uint64_t* keys_out, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  ca_status st = check_shard(q, K, dtype, B, L_shard, pos0, L, Hq, Hkv, d, W,
+                             k, W_i, workspace);
+  if (st != CA_OK) return st;
+  if (!keys_out && k > 0) return CA_ERR_INVALID_ARG;
+  if (keys_out && !aligned16(keys_out)) return CA_ERR_ALIGNMENT;
+  if (dtype != CA_BF16) return CA_ERR_UNSUPPORTED;  // tensor-core pass only
+  if (workspace_bytes < decode_ws(B, L_shard, Hq, Hkv, k))
+    return CA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t cleared = ca::kStatusBytes + decode_claims_bytes(B, Hkv);
+  if (cudaMemsetAsync(workspace, 0, cleared, s) != cudaSuccess)
+    return CA_ERR_CUDA;
+  ca::DecodeArgs a;
+  shard_args(a, q, K, K, B, L_shard, pos0, L, Hq, Hkv, W, k, W_i, workspace);
+  a.mode = ca::kShardSelect;
+  a.keys_out = keys_out;
+  a.nchunks = ca::decode_chunks(B, L_shard, Hkv, k);
+  a.chunk_len = ca::decode_chunk_len(L_shard, a.nchunks);
+  a.cand = (uint64_t*)((char*)workspace + cleared);
+  if (k == 0) return CA_OK;  // nothing to select: keys_out is empty
+  return launch_status(ca::decode_launch(a, true, d, s));
+}
+
+ca_status condensate_attn_decode_shard_attend(
+    const void* q, const void* K, const void* V, ca_dtype dtype, int B,
+    int L_shard, int pos0, int L, int Hq, int Hkv, int d, int W, int k,
+    const int32_t* W_i, const uint64_t* keys_all, int P, float* partial,
+    int32_t* idx, int32_t* idx_count, int C_max, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  ca_status st = check_shard(q, K, dtype, B, L_shard, pos0, L, Hq, Hkv, d, W,
+                             k, W_i, workspace);
+  if (st != CA_OK) return st;
+  if (!V || !partial || !idx || !idx_count || (k > 0 && !keys_all) || P < 1 ||
+      C_max < 1)
+    return CA_ERR_INVALID_ARG;
+  if (!W_i) {
+    long long need = 1LL + W + k;
+    if (need > L) need = L;
+    if (C_max < need) return CA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(V) || !aligned16(partial) || !aligned16(idx) ||
+      !aligned16(idx_count) || (keys_all && !aligned16(keys_all)))
+    return CA_ERR_ALIGNMENT;
+  if ((long long)P * (k > 0 ? k : 1) > ca::kDecodeMaxMerge)
+    return CA_ERR_UNSUPPORTED;
+  if (workspace_bytes < ca::kStatusBytes) return CA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, ca::kStatusBytes, s) != cudaSuccess)
+    return CA_ERR_CUDA;
+  ca::DecodeArgs a;
+  shard_args(a, q, K, V, B, L_shard, pos0, L, Hq, Hkv, W, k, W_i, workspace);
+  a.mode = ca::kShardAttend;
+  a.partial = partial;
+  a.idx = idx; a.idx_count = idx_count; a.C_max = C_max;
+  a.nchunks = P;
+  a.chunk_len = 0;
+  a.cand = const_cast<uint64_t*>(keys_all);
+  a.list_stride = (size_t)B * Hq * k;  // shard p's keys: keys_all[p][b][h]
+  a.head_stride = (size_t)k;
+  return launch_status(ca::decode_launch(a, dtype == CA_BF16, d, s));
+}
+
+ca_status condensate_attn_decode_shard_combine(const float* partials, int P,
+                                               int B, int Hq, int d, void* O,
+                                               ca_dtype o_dtype,
+                                               void* stream) {
+  if (!partials || !O || P < 1 || B < 1 || Hq < 1) return CA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return CA_ERR_UNSUPPORTED;
+  if (o_dtype != CA_F32 && o_dtype != CA_BF16) return CA_ERR_UNSUPPORTED;
+  if (!aligned16(partials) || !aligned16(O)) return CA_ERR_ALIGNMENT;
+  return launch_status(ca::decode_shard_combine_launch(
+      partials, P, B * Hq, d, O, o_dtype == CA_BF16, (cudaStream_t)stream));
 }
 
 ca_status condensate_attn_decode(const void* q, const void* K, const void* V,

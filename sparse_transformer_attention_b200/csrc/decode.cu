@@ -455,17 +455,17 @@ __device__ __forceinline__ void list_top_r(const uint64_t* lst, int k, int r,
 }
 
 // One warp: the m-th largest of the leading r keys of each list in src
-// (list c starts at src[c * k]; n = lists * r <= 32 * NPL), or 1 when at
-// most m of them are nonzero.
+// (list c starts at src[c * stride]; n = lists * r <= 32 * NPL), or 1 when
+// at most m of them are nonzero.
 template <int NPL>
-__device__ __forceinline__ uint64_t warp_kth_lead(const uint64_t* src, int k,
-                                                  int r, int n, int m,
-                                                  int lane) {
+__device__ __forceinline__ uint64_t warp_kth_lead(const uint64_t* src,
+                                                  size_t stride, int r, int n,
+                                                  int m, int lane) {
   uint64_t v[NPL];
 #pragma unroll
   for (int t = 0; t < NPL; ++t) {
     const int e = t * 32 + lane;
-    v[t] = e < n ? src[(size_t)(e / r) * k + e % r] : 0ull;
+    v[t] = e < n ? src[(size_t)(e / r) * stride + e % r] : 0ull;
   }
   return warp_kth<NPL>(v, m);
 }
@@ -506,24 +506,41 @@ decode_merge_attend(DecodeArgs a) {
   const int lane = tid & 31, warp = tid >> 5;
   const int gtid = tid & 255, gw = warp & 7;
   const int g = h / (a.Hq / a.Hkv);
-  const int64_t L = a.L, i = L - 1;
-  const int Wb = row_window(a.W_i, b, a.W_h, h, a.W, (int)L, a.status,
+  // this cache holds the sequence positions [p0, p1); the query is at i
+  const int64_t L = a.L, i = (int64_t)a.Lg - 1;
+  const int64_t p0 = a.pos0, p1 = p0 + L;
+  const bool select_only = a.mode == kShardSelect;
+  const bool shard_part = a.mode == kShardAttend;
+  const int Wb = row_window(a.W_i, b, a.W_h, h, a.W, a.Lg, a.status,
                             tid == 0);
   const int kh = head_k(a.k_h, h, k, a.status, tid == 0);
   const bool want_mass = a.mass != nullptr || a.lse != nullptr;
   const int64_t lo = (i - Wb + 1) > 0 ? (i - Wb + 1) : 0;
   const int64_t ncand_pos = (i - Wb) > 0 ? (i - Wb) : 0;  // |[1, i-W]|
-  const int m = (int)(kh < ncand_pos ? kh : ncand_pos);
+  // selected keys: m of the sequence's candidates, or, when selecting for
+  // one shard, of the candidates in this cache
+  const int64_t ncand_here =
+      select_only ? max((int64_t)0, min(i - Wb, p1 - 1) - max((int64_t)1, p0) + 1)
+                  : ncand_pos;
+  const int m = (int)(kh < ncand_here ? kh : ncand_here);
   const int anc = lo > 0 ? 1 : 0;
   const int64_t count = anc + m + (i - lo + 1);
+  // the anchor and window rows in this cache: the anchor when p0 = 0, then
+  // positions [wlo, whi]
+  const int anc_here = (anc && p0 == 0) ? 1 : 0;
+  const int64_t wlo = lo > p0 ? lo : p0, whi = i < p1 - 1 ? i : p1 - 1;
+  const int64_t nwin_here =
+      select_only ? 0 : anc_here + (whi >= wlo ? whi - wlo + 1 : 0);
 
   const T* qh = reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + h) * D;
   float qv[DL];
   load_f32<T, DL>(qh + lane * DL, qv);
+  // row r of this cache is sequence position p0 + r
   const T* Kg = reinterpret_cast<const T*>(a.K) +
                 ((size_t)b * a.Hkv + g) * (size_t)L * D + lane * DL;
   const T* Vg = reinterpret_cast<const T*>(a.V) +
                 ((size_t)b * a.Hkv + g) * (size_t)L * D + lane * DL;
+  auto row_of = [&](int64_t j) -> size_t { return (size_t)(j - p0) * D; };
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e)/sqrt(d)
   Online<DL> acc;
   {
@@ -531,13 +548,13 @@ decode_merge_attend(DecodeArgs a) {
     // once, so that the window gathers below wait for one L2 round trip
     // rather than one HBM round trip per batch of rows
     constexpr int kLines = D * (int)sizeof(T) / 128;
-    const int64_t nwin = min(anc + (i - lo + 1), (int64_t)512);
+    const int64_t nwin = min(nwin_here, (int64_t)512);
     const char* kb = reinterpret_cast<const char*>(Kg - lane * DL);
     const char* vb = reinterpret_cast<const char*>(Vg - lane * DL);
     for (int64_t e = tid; e < nwin * kLines; e += kMergeThreads) {
       const int64_t row = e / kLines, ln = e % kLines;
-      const int64_t j = (anc && row == 0) ? 0 : lo + (row - anc);
-      const size_t o = (size_t)j * D * sizeof(T) + (size_t)ln * 128;
+      const int64_t j = (anc_here && row == 0) ? 0 : wlo + (row - anc_here);
+      const size_t o = row_of(j) * sizeof(T) + (size_t)ln * 128;
       asm volatile("prefetch.global.L2 [%0];" ::"l"(kb + o));
       asm volatile("prefetch.global.L2 [%0];" ::"l"(vb + o));
     }
@@ -545,18 +562,20 @@ decode_merge_attend(DecodeArgs a) {
 
   if (warp >= 8) {
     // ---------------- anchor and window rows (no dependence on selection;
-    // they run while the score grid drains)
-    const int64_t nwin = anc + (i - lo + 1);
+    // they run while the score grid drains).  A shard selection attends to
+    // nothing: these warps leave before any CTA-wide barrier.
+    if (select_only) return;
+    const int64_t nwin = nwin_here;
 #pragma unroll 1
     for (int64_t e0 = gw; e0 < nwin; e0 += 8 * UG) {
       float kf[UG][DL], vf[UG][DL];
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
         const int64_t e = e0 + 8 * u;
-        int64_t j = 0;
-        if (e < nwin) j = (anc && e == 0) ? 0 : lo + (e - anc);
-        load_f32<T, DL>(Kg + (size_t)j * D, kf[u]);
-        load_f32<T, DL>(Vg + (size_t)j * D, vf[u]);
+        int64_t j = p0;
+        if (e < nwin) j = (anc_here && e == 0) ? 0 : wlo + (e - anc_here);
+        load_f32<T, DL>(Kg + row_of(j), kf[u]);
+        load_f32<T, DL>(Vg + row_of(j), vf[u]);
       }
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
@@ -594,13 +613,20 @@ decode_merge_attend(DecodeArgs a) {
     // The lists are written by the score kernel, which may still be
     // finishing: wait for it (programmatic dependent launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * ncand;
+    // list c of this q-head: k keys at src + c * list_stride (the workspace
+    // lists of the score pass, or every shard's keys)
+    const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * a.head_stride;
+    const size_t lstride = a.list_stride;
     // every list into shared memory at once: 16-byte asynchronous copies
-    // (the list area of a head starts 16-byte aligned: k keys per list,
-    // 8 bytes each, and the workspace lists start at a 256-byte boundary;
-    // an odd k leaves the head's area 8-byte aligned: then plain loads)
-    const bool async_ok = (((uintptr_t)src) & 15u) == 0;
-    if (async_ok) {
+    // when the lists are contiguous (the list area of a head starts 16-byte
+    // aligned: k keys per list, 8 bytes each, and the workspace lists start
+    // at a 256-byte boundary; an odd k leaves the head's area 8-byte
+    // aligned: then plain loads)
+    const bool async_ok = lstride == (size_t)k && (((uintptr_t)src) & 15u) == 0;
+    if (lstride != (size_t)k) {
+      for (int e = gtid; e < ncand; e += 256)
+        cand[e] = src[(size_t)(e / k) * lstride + e % k];
+    } else if (async_ok) {
       for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                          (uint32_t)__cvta_generic_to_shared(cand + e)),
@@ -624,8 +650,9 @@ decode_merge_attend(DecodeArgs a) {
     const bool use_floor = fast && m > 0 && r <= kDecodeTopR && nt <= 512;
     const bool lead = use_floor && a.top_first;
     if (lead && gw == 0) {
-      const uint64_t F = nt <= 128 ? warp_kth_lead<4>(src, k, r, nt, m, lane)
-                                   : warp_kth_lead<16>(src, k, r, nt, m, lane);
+      const uint64_t F = nt <= 128
+                             ? warp_kth_lead<4>(src, lstride, r, nt, m, lane)
+                             : warp_kth_lead<16>(src, lstride, r, nt, m, lane);
       if (lane == 0) s_T = F;
     }
     if (async_ok) asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -728,8 +755,25 @@ decode_merge_attend(DecodeArgs a) {
         }
       }
       MergeBar::sync();
-      // ascending positions: each selected key goes to its rank
       const int got = min(min(s_m, m), 128);
+      if (select_only) {
+        // the shard's best keys, largest first (so that a list's leading
+        // keys are its best), 0 after them
+        uint64_t* out = a.keys_out + ((size_t)b * a.Hq + h) * k;
+        auto key_of = [](uint64_t pr) {
+          return make_key(__uint_as_float((uint32_t)pr), (uint32_t)(pr >> 32));
+        };
+        if (gtid < got) {
+          const uint64_t my = key_of(pairs[gtid]);
+          int rank = 0;
+          for (int e = 0; e < got; ++e) rank += key_of(pairs[e]) > my;
+          out[rank] = my;
+        }
+        for (int e = got + gtid; e < k; e += 256) out[e] = 0ull;
+        if (m > 0 && s_m != m && gtid == 0) raise_flag(a.status, kErrInternal);
+        return;
+      }
+      // ascending positions: each selected key goes to its rank
       if (gtid < got) {
         const uint64_t my = pairs[gtid];
         int rank = 0;
@@ -775,6 +819,24 @@ decode_merge_attend(DecodeArgs a) {
       MergeBar::sync();
       cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T, st,
                                               gtid);
+      if (select_only) {
+        // the shard's best keys, in no particular order, 0 after them
+        uint64_t* out = a.keys_out + ((size_t)b * a.Hq + h) * k;
+        if (m > 0) {
+          for (int e = gtid; e < s_n; e += 256) {
+            const uint64_t key = cand[e];
+            if (key >= s_T && key != 0ull) {
+              const int p = atomicAdd(&s_m, 1);
+              if (p < m) out[p] = key;
+              else raise_flag(a.status, kErrInternal);
+            }
+          }
+        }
+        MergeBar::sync();
+        for (int e = min(s_m, m) + gtid; e < k; e += 256) out[e] = 0ull;
+        if (m > 0 && s_m != m && gtid == 0) raise_flag(a.status, kErrInternal);
+        return;
+      }
       if (m > 0) {
         for (int e = gtid; e < s_n; e += 256) {
           const uint64_t key = cand[e];
@@ -796,21 +858,23 @@ decode_merge_attend(DecodeArgs a) {
   const int got = s_m < m ? s_m : m;
   if (m > 0 && s_m != m && tid == 0) raise_flag(a.status, kErrInternal);
   // Top-k rows, spread over all warps: the score travels with the key, so
-  // only V is read
+  // only V is read (of the rows in this cache)
 #pragma unroll 1
   for (int e0 = warp; e0 < got; e0 += NW * UG) {
     float vf[UG][DL];
 #pragma unroll
     for (int u = 0; u < UG; ++u) {
       const int e = e0 + NW * u;
-      const uint32_t j = e < got ? topj[e] : 0u;
-      load_f32<T, DL>(Vg + (size_t)j * D, vf[u]);
+      int64_t j = e < got ? (int64_t)topj[e] : p0;
+      if (j < p0 || j >= p1) j = p0;
+      load_f32<T, DL>(Vg + row_of(j), vf[u]);
     }
 #pragma unroll
     for (int u = 0; u < UG; ++u) {
       const int e = e0 + NW * u;
       if (e >= got) break;  // warp-uniform
-      acc.add(tops[e] * sl2, vf[u]);
+      const int64_t j = topj[e];
+      if (j >= p0 && j < p1) acc.add(tops[e] * sl2, vf[u]);
     }
   }
   if (lane == 0) {
@@ -834,8 +898,20 @@ decode_merge_attend(DecodeArgs a) {
       l += s_lw[w] * c;
       o += s_ow[w][dd] * c;
     }
-    TO* out = reinterpret_cast<TO*>(a.O) + ((size_t)b * a.Hq + h) * D;
-    store_out<TO>(out + dd, o / l);
+    if (shard_part) {
+      // this shard's softmax state over its part of C_i: (max, sum, o) in
+      // the log2 domain, o not yet divided by the sum (max = -inf, sum = 0
+      // when no member of C_i lies here)
+      float* pt = a.partial + ((size_t)b * a.Hq + h) * (D + 2);
+      if (dd == 0) {
+        pt[0] = M;
+        pt[1] = l;
+      }
+      pt[2 + dd] = o;
+    } else {
+      TO* out = reinterpret_cast<TO*>(a.O) + ((size_t)b * a.Hq + h) * D;
+      store_out<TO>(out + dd, o / l);
+    }
   }
   if (want_mass && tid == 32 + D) {
     // masses over the full causal softmax: C (all warps), window + anchor
@@ -864,6 +940,32 @@ decode_merge_attend(DecodeArgs a) {
   if (tid == 0) a.idx_count[(size_t)b * a.Hq + h] = (int32_t)count;
 }
 
+
+// Sequence-sharded decode, last step: combine the shards' softmax states
+// (max, sum, o) into O = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M),
+// M = max_p m_p over the shards that hold members of C_i.  One CTA per
+// (batch, q-head), one thread per output dimension.
+template <typename TO>
+__global__ void decode_shard_combine(const float* parts, int P, int rows,
+                                     int D, void* O) {
+  const int row = blockIdx.x, dd = threadIdx.x;
+  if (dd >= D) return;
+  float M = -INFINITY;
+  for (int p = 0; p < P; ++p) {
+    const float* pt = parts + ((size_t)p * rows + row) * (D + 2);
+    if (pt[1] > 0.f) M = fmaxf(M, pt[0]);
+  }
+  float l = 0.f, o = 0.f;
+  for (int p = 0; p < P; ++p) {
+    const float* pt = parts + ((size_t)p * rows + row) * (D + 2);
+    if (pt[1] > 0.f) {
+      const float c = exp2f(pt[0] - M);
+      l += pt[1] * c;
+      o += pt[2 + dd] * c;
+    }
+  }
+  store_out<TO>(reinterpret_cast<TO*>(O) + (size_t)row * D + dd, o / l);
+}
 
 // Shared memory of the score kernel: a K staging ring of 2..kMaxStages
 // stages and per-list candidate buffers of k + kSub + slack keys.  Prefer
@@ -895,13 +997,21 @@ void score_smem(int k, int* cap, int* nstages, size_t* bytes) {
 template <typename T, int D, int G>
 cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
   a.top_first = 0;
+  if (a.mode == kShardAttend) {
+    // the lists are the shards' selections, best keys first when k <= 128
+    a.top_first = a.kpow2 <= 128;
+  } else {
+    a.list_stride = (size_t)a.k;
+    a.head_stride = (size_t)a.nchunks * a.k;
+  }
   size_t smem1;
   score_smem<T, D, G>(a.k, &a.cap, &a.nstages, &smem1);
   cudaError_t e = cudaSuccess;
   const bool mass = a.mass != nullptr || a.lse != nullptr;
   // with k = 0 the set is anchor and window only: the score pass runs only
-  // for the mass reports (the candidates' sums)
-  if (a.k > 0 || mass) {
+  // for the mass reports (the candidates' sums); a shard's attend step has
+  // its lists already
+  if (a.mode != kShardAttend && (a.k > 0 || mass)) {
     bool done = false;
     if constexpr (sizeof(T) == 2) {
       // bf16: the dot products on the tensor pipe
@@ -913,6 +1023,8 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
       }
     }
     if (!done) {
+      // the CUDA-core pass scores a whole cache only
+      if (a.mode == kShardSelect) return cudaErrorNotSupported;
       auto k1 = mass ? decode_score_topk<T, D, G, true>
                      : decode_score_topk<T, D, G, false>;
       // the largest shared-memory carve-out, so that two CTAs fit per SM
@@ -983,6 +1095,18 @@ int decode_chunk_len(int L, int nchunks) {
   // a whole number of 128-key tiles of the tensor-core score pass
   int len = (L + nchunks - 1) / nchunks;
   return (len + 127) / 128 * 128;
+}
+
+cudaError_t decode_shard_combine_launch(const float* parts, int P, int rows,
+                                        int d, void* O, bool o_bf16,
+                                        cudaStream_t s) {
+  prof_before(s, "decode_shard_combine");
+  if (o_bf16)
+    decode_shard_combine<__nv_bfloat16><<<rows, d, 0, s>>>(parts, P, rows, d, O);
+  else
+    decode_shard_combine<float><<<rows, d, 0, s>>>(parts, P, rows, d, O);
+  prof_after(s);
+  return cudaGetLastError();
 }
 
 cudaError_t decode_launch(const DecodeArgs& a, bool bf16, int d,

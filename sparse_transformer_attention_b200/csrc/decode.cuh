@@ -19,11 +19,27 @@ constexpr int kDecodeMaxMerge = 8192;
 // its r = ceil(m / workers) best keys when r is at most this.
 constexpr int kDecodeTopR = 8;
 
+// What the merge launch does with the exact Top-k it selects.
+enum DecodeMode {
+  kDecodeAttend = 0,  // attend over C_i and write O (the whole cache here)
+  kShardSelect = 1,   // write the shard's best keys to keys_out, no attend
+  kShardAttend = 2,   // lists are every shard's keys; attend over the part
+                      // of C_i in this shard and write the partial state
+};
+
 struct DecodeArgs {
   const void* q;
   const void* K;
   const void* V;
   int B, L, Hq, Hkv, W, k;
+  int Lg;               // cache length of the whole sequence (L unless the
+                        // cache is sharded along L); the query is at Lg - 1
+  int pos0;             // position of this cache's row 0 in the sequence
+  int mode;             // DecodeMode
+  uint64_t* keys_out;   // kShardSelect: [B, Hq, k] best keys of the shard
+  float* partial;       // kShardAttend: [B, Hq, d + 2] = (max, sum, o[d])
+  size_t list_stride;   // keys between consecutive lists of a q-head
+  size_t head_stride;   // keys between the lists of consecutive q-heads
   const int32_t* W_i;   // [B] or NULL
   const int32_t* W_h;   // [Hq] or NULL
   const int32_t* k_h;   // [Hq] or NULL
@@ -57,5 +73,9 @@ cudaError_t decode_score_tc_launch(const DecodeArgs& a, int d, bool mass,
 int decode_chunk_len(int L, int nchunks);
 cudaError_t decode_launch(const DecodeArgs& a, bool bf16, int d,
                           cudaStream_t stream);
+// O[row] from the P shards' (max, sum, o[d]) states parts[P, rows, d + 2].
+cudaError_t decode_shard_combine_launch(const float* parts, int P, int rows,
+                                        int d, void* O, bool o_bf16,
+                                        cudaStream_t stream);
 
 }  // namespace ca

@@ -173,14 +173,16 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   const int worker = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int nworkers = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int L = a.L;
+  const int L = a.L;        // rows of this cache (a shard of the sequence)
+  const int pos0 = a.pos0;  // sequence position of row 0
   if (tid == 0) {
-    // per q-head of the group: last candidate position and Top-k size
+    // per q-head of the group: last candidate position (in the sequence,
+    // whose query sits at Lg - 1) and Top-k size
     for (int h = 0; h < G; ++h) {
       const int hq = g * G + h;
       const bool rep = worker == 0;
-      sh->hi[h] = (L - 1) - row_window(a.W_i, b, a.W_h, hq, a.W, L, a.status,
-                                       rep);
+      sh->hi[h] = (a.Lg - 1) - row_window(a.W_i, b, a.W_h, hq, a.W, a.Lg,
+                                          a.status, rep);
       sh->kk[h] = head_k(a.k_h, hq, a.k, a.status, rep);
       sh->cnt[h] = 0;
       sh->thr[h] = sh->kk[h] > 0 ? 0ull : ~0ull;  // k = 0 admits nothing
@@ -213,10 +215,11 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
   int hi = -1;
 #pragma unroll
   for (int h = 0; h < G; ++h) hi = max(hi, sh->hi[h]);
-  // the group's candidate keys are positions 1..hi, in units of kUnitKeys
-  // keys from position 0 (position 0 and those past a head's window start
-  // are masked by the selectors)
-  const int nunits = hi >= 1 ? (hi + kUnitKeys) / kUnitKeys : 0;
+  // the group's candidate keys are positions 1..hi; in this cache, rows
+  // 0..hl, in units of kUnitKeys rows from row 0 (position 0 and positions
+  // past a head's window start are masked by the selectors)
+  const int hl = min(hi - pos0, L - 1);
+  const int nunits = (hi >= 1 && hl >= 0) ? (hl + kUnitKeys) / kUnitKeys : 0;
   volatile int* abort_flag = &sh->abort;
 
   if (warp == 0) {
@@ -416,8 +419,8 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         sm100::tc_fence_before();
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&sh->tempty[tb]);
-        const int j = pos + kq;
-        const bool in = j >= 1 && j <= hi;
+        const int j = pos0 + pos + kq;  // sequence position
+        const bool in = pos + kq <= hl && j >= 1;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float sc = __uint_as_float(v[h]);
@@ -485,7 +488,10 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
             a.cand + (((size_t)b * a.Hq + (size_t)g * G + h) * a.nchunks +
                       worker) * a.k;
         const int cnt = sh->cnt[h];
-        const int mh = min(sh->kk[h], max(hi_h[h], 0));
+        // the head's candidates in this cache: positions max(1, pos0) ..
+        // min(hi_h, pos0 + L - 1)
+        const int nc = max(0, min(hi_h[h], pos0 + L - 1) - max(1, pos0) + 1);
+        const int mh = min(sh->kk[h], nc);
         const int r = mh > 0 ? (mh + nworkers - 1) / nworkers : 0;
         uint64_t v[4];
 #pragma unroll

@@ -34,7 +34,7 @@ def test_header_lists_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     for name in header_functions():
         assert hasattr(lib, name), name
-    assert lib.condensate_attn_version() == 200
+    assert lib.condensate_attn_version() == 300
 
 
 def test_status_strings(lib):
@@ -116,6 +116,71 @@ def test_invalid_arguments_rejected_before_launch(lib, call, over, code):
     key_map = {"q": "Q", "L": "n"} if call is _prefill else {}
     over = {key_map.get(k, k): v for k, v in over.items()}
     assert call(lib, **over) == code
+
+
+def _select(lib, **over):
+    a = dict(q=FAKE, K=FAKE, dtype=1, B=1, Ls=500, pos0=0, L=1000, Hq=8,
+             Hkv=2, d=128, W=64, k=16, keys=FAKE, ws=FAKE, ws_bytes=16)
+    a.update(over)
+    P = ctypes.c_void_p
+    return lib.condensate_attn_decode_shard_select(
+        P(a["q"]), P(a["K"]), a["dtype"], a["B"], a["Ls"], a["pos0"], a["L"],
+        a["Hq"], a["Hkv"], a["d"], a["W"], a["k"], None, P(a["keys"]),
+        P(a["ws"]) if a["ws"] else None, a["ws_bytes"], None)
+
+
+def _attend(lib, **over):
+    a = dict(q=FAKE, K=FAKE, V=FAKE, dtype=1, B=1, Ls=500, pos0=500, L=1000,
+             Hq=8, Hkv=2, d=128, W=64, k=16, keys=FAKE, P=2, part=FAKE,
+             idx=FAKE, cnt=FAKE, C_max=81, ws=FAKE, ws_bytes=16)
+    a.update(over)
+    P = ctypes.c_void_p
+    return lib.condensate_attn_decode_shard_attend(
+        P(a["q"]), P(a["K"]), P(a["V"]), a["dtype"], a["B"], a["Ls"],
+        a["pos0"], a["L"], a["Hq"], a["Hkv"], a["d"], a["W"], a["k"], None,
+        P(a["keys"]) if a["keys"] else None, a["P"],
+        P(a["part"]) if a["part"] else None, P(a["idx"]), P(a["cnt"]),
+        a["C_max"], P(a["ws"]) if a["ws"] else None, a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("call,over,code", [
+    (_select, {"pos0": 501}, binding.CA_ERR_INVALID_ARG),   # past the end
+    (_select, {"pos0": -1}, binding.CA_ERR_INVALID_ARG),
+    (_select, {"Ls": 0}, binding.CA_ERR_INVALID_ARG),
+    (_select, {"keys": 0}, binding.CA_ERR_INVALID_ARG),
+    (_select, {"q": 0}, binding.CA_ERR_INVALID_ARG),
+    (_select, {"dtype": 0}, binding.CA_ERR_UNSUPPORTED),    # bf16 only
+    (_select, {"d": 96}, binding.CA_ERR_UNSUPPORTED),
+    (_select, {"keys": FAKE + 8}, binding.CA_ERR_ALIGNMENT),
+    (_select, {"ws": 0}, binding.CA_ERR_WORKSPACE),
+    (_select, {}, binding.CA_ERR_WORKSPACE),                # 16 bytes
+    (_attend, {"pos0": 501}, binding.CA_ERR_INVALID_ARG),
+    (_attend, {"P": 0}, binding.CA_ERR_INVALID_ARG),
+    (_attend, {"keys": 0}, binding.CA_ERR_INVALID_ARG),
+    (_attend, {"part": 0}, binding.CA_ERR_INVALID_ARG),
+    (_attend, {"C_max": 80}, binding.CA_ERR_INVALID_ARG),
+    (_attend, {"P": 1024}, binding.CA_ERR_UNSUPPORTED),     # P k > 8192
+    (_attend, {"part": FAKE + 4}, binding.CA_ERR_ALIGNMENT),
+    (_attend, {}, binding.CA_ERR_WORKSPACE),                # 16 bytes
+])
+def test_shard_arguments_rejected_before_launch(lib, call, over, code):
+    assert call(lib, **over) == code
+
+
+def test_shard_combine_arguments(lib):
+    P = ctypes.c_void_p
+    f = lib.condensate_attn_decode_shard_combine
+    assert f(P(FAKE), 0, 1, 8, 128, P(FAKE), 0, None) == \
+        binding.CA_ERR_INVALID_ARG
+    assert f(None, 2, 1, 8, 128, P(FAKE), 0, None) == \
+        binding.CA_ERR_INVALID_ARG
+    assert f(P(FAKE), 2, 1, 8, 96, P(FAKE), 0, None) == \
+        binding.CA_ERR_UNSUPPORTED
+    assert f(P(FAKE + 8), 2, 1, 8, 128, P(FAKE), 0, None) == \
+        binding.CA_ERR_ALIGNMENT
+    ws = lib.condensate_attn_decode_shard_workspace_size
+    assert ws(1, 1, 65536, 32, 8, 128, 64) > 256
+    assert ws(1, 1, 0, 32, 8, 128, 64) == 0
 
 
 def test_k_limits(lib):
