@@ -28,7 +28,7 @@
  * q-head h reads kv-head h / (Hq/Hkv) (grouped-query attention).
  * idx rows hold C_i in ascending order, padded with -1 up to C_max.
  * Supported: d in {64, 128}; dtype CA_F32 or CA_BF16 for Q/K/V (all three
- * alike); O may be CA_F32 or CA_BF16; Hq/Hkv in {1, 2, 4, 8}; k <= 64 for
+ * alike); O may be CA_F32 or CA_BF16; Hq/Hkv in {1, 2, 4, 8}; k <= 128 for
  * prefill and k <= 1024 for decode (CA_ERR_UNSUPPORTED beyond).
  * Scores and the softmax are accumulated in fp32; selection uses the
  * unscaled fp32 dot product with the tie rule above.

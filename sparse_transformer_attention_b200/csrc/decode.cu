@@ -18,11 +18,11 @@
 // of the lists contains the global Top-k, since every global Top-k member
 // is among the best k of its own chunk.
 //
-// Launch 2, decode_merge_attend: grid (Hq, B).  Half of each CTA gathers the
+// Launch 2, decode_merge_attend: grid (Hq, B).  Every warp first gathers
 // anchor and window rows into its fp32 online softmax while the score grid
-// drains (they do not depend on the selection); the other half merges the
-// lists into the exact Top-k (for k <= 128: a floor from each list's best
-// few keys, the exact m-th best of the keys at or above it, ranks for
+// drains (they do not depend on the selection); then half of the CTA merges
+// the lists into the exact Top-k (for k <= 128: a floor from each list's
+// best few keys, the exact m-th best of the keys at or above it, ranks for
 // ascending positions; else a radix select); then all warps accumulate the
 // Top-k rows, whose scores come with their keys, and the per-warp softmax
 // states are combined.
@@ -435,6 +435,48 @@ struct Online {
   }
 };
 
+// How many of a[beg..end) exceed x: eight independent loads per step, so
+// that one thread's count is not a chain of dependent shared-memory reads.
+__device__ __forceinline__ int count_above(const uint64_t* a, int beg, int end,
+                                           uint64_t x) {
+  int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+  int f = beg;
+#pragma unroll 1
+  for (; f + 8 <= end; f += 8) {
+    const uint64_t v0 = a[f], v1 = a[f + 1], v2 = a[f + 2], v3 = a[f + 3];
+    const uint64_t v4 = a[f + 4], v5 = a[f + 5], v6 = a[f + 6], v7 = a[f + 7];
+    c0 += (v0 > x) + (v4 > x);
+    c1 += (v1 > x) + (v5 > x);
+    c2 += (v2 > x) + (v6 > x);
+    c3 += (v3 > x) + (v7 > x);
+  }
+#pragma unroll 1
+  for (; f < end; ++f) c0 += a[f] > x;
+  return c0 + c1 + c2 + c3;
+}
+
+// How many keys of a[0..n) have a position below j (the same eight-wide
+// steps as count_above).
+__device__ __forceinline__ int count_pos_below(const uint64_t* a, int n,
+                                               uint32_t j) {
+  int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+  int f = 0;
+#pragma unroll 1
+  for (; f + 8 <= n; f += 8) {
+    const uint32_t v0 = key_index(a[f]), v1 = key_index(a[f + 1]);
+    const uint32_t v2 = key_index(a[f + 2]), v3 = key_index(a[f + 3]);
+    const uint32_t v4 = key_index(a[f + 4]), v5 = key_index(a[f + 5]);
+    const uint32_t v6 = key_index(a[f + 6]), v7 = key_index(a[f + 7]);
+    c0 += (v0 < j) + (v4 < j);
+    c1 += (v1 < j) + (v5 < j);
+    c2 += (v2 < j) + (v6 < j);
+    c3 += (v3 < j) + (v7 < j);
+  }
+#pragma unroll 1
+  for (; f < n; ++f) c0 += key_index(a[f]) < j;
+  return c0 + c1 + c2 + c3;
+}
+
 // The r best keys of one worker list lst[0..k) (k <= 128, read by one warp)
 // to out[0..r), largest first, 0 once the list runs out.
 __device__ __forceinline__ void list_top_r(const uint64_t* lst, int k, int r,
@@ -454,32 +496,6 @@ __device__ __forceinline__ void list_top_r(const uint64_t* lst, int k, int r,
   }
 }
 
-// One warp: the m-th largest of the leading r keys of each list in src
-// (list c starts at src[c * stride]; n = lists * r <= 32 * NPL), or 1 when
-// at most m of them are nonzero.
-template <int NPL>
-__device__ __forceinline__ uint64_t warp_kth_lead(const uint64_t* src,
-                                                  size_t stride, int r, int n,
-                                                  int m, int lane) {
-  uint64_t v[NPL];
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    const int e = t * 32 + lane;
-    v[t] = e < n ? src[(size_t)(e / r) * stride + e % r] : 0ull;
-  }
-  return warp_kth<NPL>(v, m);
-}
-
-// One warp: the m-th largest of the n keys in src (n <= 32 * NPL), or 1
-// when at most m are nonzero.
-template <int NPL>
-__device__ __forceinline__ uint64_t warp_kth_of(const uint64_t* src, int n,
-                                                int m, int lane) {
-  uint64_t v[NPL];
-  warp_load_keys<NPL>(src, n, v, lane);
-  return warp_kth<NPL>(v, m);
-}
-
 template <typename T, int D, typename TO>
 __global__ void __launch_bounds__(kMergeThreads)
 decode_merge_attend(DecodeArgs a) {
@@ -495,11 +511,12 @@ decode_merge_attend(DecodeArgs a) {
   uint32_t* topj = reinterpret_cast<uint32_t*>(pairs + 128);    // [kpow2]
   float* tops = reinterpret_cast<float*>(topj + a.kpow2);       // [kpow2]
   SelectState<1>* st = reinterpret_cast<SelectState<1>*>(tops + a.kpow2);
+  int* s_cnt = reinterpret_cast<int*>(st + 1);                  // [512]
   __shared__ int s_n, s_kk, s_m;
   __shared__ uint64_t s_T, s_t0[8];
   __shared__ float s_mw[NW], s_lw[NW];
   __shared__ float s_ow[NW][D];
-  __shared__ float s_wm[8], s_wl[8], s_s0;  // window+anchor states; anchor score
+  __shared__ float s_wm[NW], s_wl[NW], s_s0;  // window+anchor states; anchor score
   __shared__ int s_seg[8];                     // survivors per merge warp
 
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -560,18 +577,19 @@ decode_merge_attend(DecodeArgs a) {
     }
   }
 
-  if (warp >= 8) {
-    // ---------------- anchor and window rows (no dependence on selection;
-    // they run while the score grid drains).  A shard selection attends to
-    // nothing: these warps leave before any CTA-wide barrier.
-    if (select_only) return;
+  // A shard selection attends to nothing: warps 8-15 leave before any
+  // CTA-wide barrier (warps 0-7 leave after the selection).
+  if (select_only && warp >= 8) return;
+  if (!select_only) {
+    // ---------------- anchor and window rows, every warp: they do not
+    // depend on the selection, and the score grid is still draining
     const int64_t nwin = nwin_here;
 #pragma unroll 1
-    for (int64_t e0 = gw; e0 < nwin; e0 += 8 * UG) {
+    for (int64_t e0 = warp; e0 < nwin; e0 += NW * UG) {
       float kf[UG][DL], vf[UG][DL];
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
-        const int64_t e = e0 + 8 * u;
+        const int64_t e = e0 + NW * u;
         int64_t j = p0;
         if (e < nwin) j = (anc_here && e == 0) ? 0 : wlo + (e - anc_here);
         load_f32<T, DL>(Kg + row_of(j), kf[u]);
@@ -579,7 +597,7 @@ decode_merge_attend(DecodeArgs a) {
       }
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
-        if (e0 + 8 * u >= nwin) break;  // warp-uniform
+        if (e0 + NW * u >= nwin) break;  // warp-uniform
         float dot = 0.f;
 #pragma unroll
         for (int e = 0; e < DL; ++e) dot = fmaf(qv[e], kf[u][e], dot);
@@ -593,10 +611,10 @@ decode_merge_attend(DecodeArgs a) {
       // the window + anchor part alone, and the anchor's own score (inside
       // the window when the window reaches position 0)
       if (lane == 0) {
-        s_wm[gw] = acc.m;
-        s_wl[gw] = acc.l;
+        s_wm[warp] = acc.m;
+        s_wl[warp] = acc.l;
       }
-      if (gw == 0) {
+      if (warp == NW - 1) {
         float k0[DL];
         load_f32<T, DL>(Kg, k0);
         float dot = 0.f;
@@ -608,72 +626,89 @@ decode_merge_attend(DecodeArgs a) {
         if (lane == 0) s_s0 = dot * sl2;
       }
     }
-  } else {
+  }
+  if (warp < 8) {
     // ---------------- merge the worker lists into the exact Top-k
-    // The lists are written by the score kernel, which may still be
-    // finishing: wait for it (programmatic dependent launch).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     // list c of this q-head: k keys at src + c * list_stride (the workspace
     // lists of the score pass, or every shard's keys)
     const uint64_t* src = a.cand + ((size_t)b * a.Hq + h) * a.head_stride;
     const size_t lstride = a.list_stride;
-    // every list into shared memory at once: 16-byte asynchronous copies
-    // when the lists are contiguous (the list area of a head starts 16-byte
-    // aligned: k keys per list, 8 bytes each, and the workspace lists start
-    // at a 256-byte boundary; an odd k leaves the head's area 8-byte
-    // aligned: then plain loads)
     const bool async_ok = lstride == (size_t)k && (((uintptr_t)src) & 15u) == 0;
-    if (lstride != (size_t)k) {
-      for (int e = gtid; e < ncand; e += 256)
-        cand[e] = src[(size_t)(e / k) * lstride + e % k];
-    } else if (async_ok) {
-      for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                         (uint32_t)__cvta_generic_to_shared(cand + e)),
-                     "l"(src + e)
-                     : "memory");
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
-    } else {
-      for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
-    }
     // k <= 128: a floor first.  With each list's r = ceil(m / lists) best
     // keys, the m-th largest of those, F, has m keys at or above it, so the
     // global m-th best key is >= F and only keys >= F can be selected
     // (about m survive).  The tensor-core pass writes those r keys at the
-    // front of each list: then warp 0 reads them from global memory while
-    // the copies land.
+    // front of each list.  F and the exact selection among the survivors
+    // are found by ranks (a key's number of larger keys), counted by
+    // several threads per key: no barrier per step, and loops that stay
+    // rolled.
     const bool fast = a.kpow2 <= 128;
     const int r = m > 0 ? (m + a.nchunks - 1) / a.nchunks : 0;
     const int nt = a.nchunks * r;
     const bool use_floor = fast && m > 0 && r <= kDecodeTopR && nt <= 512;
     const bool lead = use_floor && a.top_first;
-    if (lead && gw == 0) {
-      const uint64_t F = nt <= 128
-                             ? warp_kth_lead<4>(src, lstride, r, nt, m, lane)
-                             : warp_kth_lead<16>(src, lstride, r, nt, m, lane);
-      if (lane == 0) s_T = F;
+    {
+      // The lists are written by the score kernel, which may still be
+      // finishing: wait for it (programmatic dependent launch).
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      // every list into shared memory at once: 16-byte asynchronous copies
+      // when the lists are contiguous (the list area of a head starts
+      // 16-byte aligned: k keys per list, 8 bytes each, and the workspace
+      // lists start at a 256-byte boundary; an odd k leaves the head's area
+      // 8-byte aligned: then plain loads)
+      if (lstride != (size_t)k) {
+        for (int e = gtid; e < ncand; e += 256)
+          cand[e] = src[(size_t)(e / k) * lstride + e % k];
+      } else if (async_ok) {
+        for (int e = 2 * gtid; e + 1 < ncand; e += 512) {
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                           (uint32_t)__cvta_generic_to_shared(cand + e)),
+                       "l"(src + e)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if ((ncand & 1) && gtid == 0) cand[ncand - 1] = src[ncand - 1];
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      } else {
+        for (int e = gtid; e < ncand; e += 256) cand[e] = src[e];
+      }
     }
-    if (async_ok) asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (gtid == 0) {
       s_n = 0;
       s_m = 0;
       s_kk = m > 0 ? m : 1;
-      if (!lead) s_T = fast ? 1ull : 0ull;  // 1: no floor, real keys only
+      s_T = fast ? 1ull : 0ull;  // 1: no floor, real keys only
     }
     MergeBar::sync();
     if (fast) {
-      // Loops stay rolled: this code runs once per CTA, from a cold
-      // instruction cache.
-      if (use_floor && !lead) {
-        for (int c = gw; c < a.nchunks; c += 8)
-          list_top_r(cand + (size_t)c * k, k, r, surv + (size_t)c * r, lane);
+      if (use_floor) {
+        // the leading keys: list c's q-th at lk[c * ls + q]
+        if (!lead) {
+          for (int c = gw; c < a.nchunks; c += 8)
+            list_top_r(cand + (size_t)c * k, k, r, surv + (size_t)c * r, lane);
+          MergeBar::sync();
+        }
+        // the nt leading keys, contiguous in surv (list_top_r wrote them so)
+        if (lead)
+          for (int e = gtid; e < nt; e += 256)
+            surv[e] = cand[(size_t)(e / r) * k + e % r];
+        for (int e = gtid; e < nt; e += 256) s_cnt[e] = 0;
         MergeBar::sync();
-        if (gw == 0) {
-          const uint64_t F = nt <= 128 ? warp_kth_of<4>(surv, nt, m, lane)
-                                       : warp_kth_of<16>(surv, nt, m, lane);
-          if (lane == 0) s_T = F;
+        // each key's rank counted in S slices of the others, by S threads
+        const int S = nt < 256 ? 256 / nt : 1;
+        const int slice = (nt + S - 1) / S;
+        for (int u = gtid; u < nt * S; u += 256) {
+          const int e = u % nt, sl = u / nt;
+          const uint64_t my = surv[e];
+          if (my == 0ull) continue;
+          const int part =
+              count_above(surv, sl * slice, min(nt, (sl + 1) * slice), my);
+          if (part) atomicAdd(&s_cnt[e], part);
+        }
+        MergeBar::sync();
+        for (int e = gtid; e < nt; e += 256) {
+          const uint64_t my = surv[e];
+          if (my != 0ull && s_cnt[e] == m - 1) s_T = my;  // m - 1 above it
         }
         MergeBar::sync();
       }
@@ -692,10 +727,12 @@ decode_merge_attend(DecodeArgs a) {
           const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
           if (keep) {
             surv[beg + w + __popc(bal & ((1u << lane) - 1u))] = key;
-            const char* row = reinterpret_cast<const char*>(
-                Vg - lane * DL + (size_t)key_index(key) * D);
-            for (int o = 0; o < D * (int)sizeof(T); o += 128)
-              asm volatile("prefetch.global.L2 [%0];" ::"l"(row + o));
+            if (!select_only) {
+              const char* row = reinterpret_cast<const char*>(
+                  Vg - lane * DL + row_of(key_index(key)));
+              for (int o = 0; o < D * (int)sizeof(T); o += 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row + o));
+            }
           }
           w += __popc(bal);
         }
@@ -709,77 +746,72 @@ decode_merge_attend(DecodeArgs a) {
           off[c] = ns;
           ns += s_seg[c];
         }
-        // survivors, contiguous, into cand (no longer read)
+        // survivor e (in segment order): segment c holds s_seg[c] keys at
+        // surv + c * per
         auto gather = [&](int e) -> uint64_t {
           int c = 0;
 #pragma unroll
           for (int q = 1; q < 8; ++q) c = e >= off[q] ? q : c;
           return surv[(size_t)c * per + (e - off[c])];
         };
+        // the survivors, contiguous, into cand (no longer read)
+        for (int e = gtid; e < ns; e += 256) {
+          cand[e] = gather(e);
+          if (e < 512) s_cnt[e] = 0;
+        }
+        if (gtid == 0) s_n = ns;
+        MergeBar::sync();
         if (ns <= 512) {
-          if (gw == 0) {
-            for (int e = lane; e < ns; e += 32) cand[e] = gather(e);
-            __syncwarp();
-            const uint64_t Tm = ns <= 128 ? warp_kth_of<4>(cand, ns, m, lane)
-                                          : warp_kth_of<16>(cand, ns, m, lane);
-            int got = 0;
-            for (int e0 = 0; e0 < ns; e0 += 32) {
-              const int e = e0 + lane;
-              const uint64_t key = e < ns ? cand[e] : 0ull;
-              const bool keep = key >= Tm;
-              const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-              const int p = got + __popc(bal & ((1u << lane) - 1u));
-              if (keep && p < 128)
-                pairs[p] = ((uint64_t)key_index(key) << 32) |
-                           __float_as_uint(key_score(key));
-              got += __popc(bal);
-            }
-            if (lane == 0) s_m = got;
+          // a survivor with fewer than m larger survivors is selected, at
+          // the slot of its rank (so pairs holds them largest first); each
+          // rank is counted by S threads over slices of the survivors
+          const int S = ns < 256 ? 256 / ns : 1;
+          const int slice = (ns + S - 1) / S;
+          for (int u = gtid; u < ns * S; u += 256) {
+            const int e = u % ns, sl = u / ns;
+            const int part = count_above(cand, sl * slice,
+                                         min(ns, (sl + 1) * slice), cand[e]);
+            if (part) atomicAdd(&s_cnt[e], part);
           }
+          MergeBar::sync();
+          for (int e = gtid; e < ns; e += 256)
+            if (s_cnt[e] < m) pairs[s_cnt[e]] = cand[e];
+          if (gtid == 0) s_m = min(ns, m);
         } else {
           // many survivors: radix select over the eight warps
-          for (int e = gtid; e < ns; e += 256) cand[e] = gather(e);
-          if (gtid == 0) s_n = ns;
-          MergeBar::sync();
           cta_select_thresholds<256, 1, MergeBar>(cand, 0, &s_n, &s_kk, &s_T,
                                                   st, gtid);
           for (int e = gtid; e < ns; e += 256) {
             const uint64_t key = cand[e];
             if (key >= s_T && key != 0ull) {
               const int p = atomicAdd(&s_m, 1);
-              if (p < 128)
-                pairs[p] = ((uint64_t)key_index(key) << 32) |
-                           __float_as_uint(key_score(key));
+              if (p < 128) pairs[p] = key;
             }
           }
         }
       }
       MergeBar::sync();
+      // pairs[0..got) holds the selected keys
       const int got = min(min(s_m, m), 128);
       if (select_only) {
         // the shard's best keys, largest first (so that a list's leading
         // keys are its best), 0 after them
         uint64_t* out = a.keys_out + ((size_t)b * a.Hq + h) * k;
-        auto key_of = [](uint64_t pr) {
-          return make_key(__uint_as_float((uint32_t)pr), (uint32_t)(pr >> 32));
-        };
         if (gtid < got) {
-          const uint64_t my = key_of(pairs[gtid]);
-          int rank = 0;
-          for (int e = 0; e < got; ++e) rank += key_of(pairs[e]) > my;
-          out[rank] = my;
+          const uint64_t my = pairs[gtid];
+          out[count_above(pairs, 0, got, my)] = my;
         }
         for (int e = got + gtid; e < k; e += 256) out[e] = 0ull;
         if (m > 0 && s_m != m && gtid == 0) raise_flag(a.status, kErrInternal);
         return;
       }
-      // ascending positions: each selected key goes to its rank
+      // ascending positions: each selected key goes to its position's rank
       if (gtid < got) {
         const uint64_t my = pairs[gtid];
-        int rank = 0;
-        for (int e = 0; e < got; ++e) rank += pairs[e] < my;
-        topj[rank] = (uint32_t)(my >> 32);
-        tops[rank] = __uint_as_float((uint32_t)my);
+        const uint32_t jm = key_index(my);
+        const int rank = count_pos_below(pairs, got, jm);
+        topj[rank] = jm;
+        tops[rank] = key_score(my);
       }
     } else {
       // Every chunk list holds its chunk's best k keys, so the largest of the
@@ -915,17 +947,18 @@ decode_merge_attend(DecodeArgs a) {
   }
   if (want_mass && tid == 32 + D) {
     // masses over the full causal softmax: C (all warps), window + anchor
-    // (warps 8..15 before the Top-k rows), and every candidate (the score
+    // (every warp before the Top-k rows), and every candidate (the score
     // pass's per-chunk sums), in one frame
     Lse2 c, wa, cand;
     for (int w = 0; w < NW; ++w) c.merge(s_mw[w], s_lw[w]);
-    for (int w = 0; w < 8; ++w) wa.merge(s_wm[w], s_wl[w]);
+    for (int w = 0; w < NW; ++w) wa.merge(s_wm[w], s_wl[w]);
     const float2* cml = a.cand_ml + ((size_t)b * a.Hq + h) * a.nchunks;
     for (int ch = 0; ch < a.nchunks; ++ch) cand.merge(cml[ch].x, cml[ch].y);
     mass_report(a.mass, a.lse, (size_t)b * a.Hq + h, c.m, c.l, wa.m, wa.l,
                 cand.m, cand.l, s_s0, anc != 0);
   }
-  __syncthreads();  // the sorted Top-k is visible
+  // the radix path's sorted Top-k must be visible to every thread
+  if (a.kpow2 > 128) __syncthreads();
   int32_t* idx_row = a.idx + ((size_t)b * a.Hq + h) * a.C_max;
   if (count > a.C_max && tid == 0) raise_flag(a.status, kErrCmax);
   const int64_t wcount = count < a.C_max ? count : a.C_max;
@@ -1039,7 +1072,7 @@ cudaError_t launch_typed(DecodeArgs a, cudaStream_t stream) {
     }
   }
   const size_t smem2 = (size_t)a.nchunks * a.k * 16 + 128 * 8 +
-                       (size_t)a.kpow2 * 8 + sizeof(SelectState<1>);
+                       (size_t)a.kpow2 * 8 + sizeof(SelectState<1>) + 512 * 4;
   dim3 grid2(a.Hq, a.B);
   auto k2 = a.o_bf16 ? decode_merge_attend<T, D, __nv_bfloat16>
                      : decode_merge_attend<T, D, float>;

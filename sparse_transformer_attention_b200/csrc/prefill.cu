@@ -1007,9 +1007,12 @@ cudaError_t launch_gather(const PrefillArgs& a, cudaStream_t s) {
   if (a.k <= 32) {
     if (a.o_bf16) gather_f32_as<T, D, __nv_bfloat16, 1>(a, grid, nt, s);
     else gather_f32_as<T, D, float, 1>(a, grid, nt, s);
-  } else {
+  } else if (a.k <= 64) {
     if (a.o_bf16) gather_f32_as<T, D, __nv_bfloat16, 2>(a, grid, nt, s);
     else gather_f32_as<T, D, float, 2>(a, grid, nt, s);
+  } else {
+    if (a.o_bf16) gather_f32_as<T, D, __nv_bfloat16, 4>(a, grid, nt, s);
+    else gather_f32_as<T, D, float, 4>(a, grid, nt, s);
   }
   prof_after(s);
   return cudaGetLastError();
@@ -1037,8 +1040,11 @@ cudaError_t launch_gather_mma(const PrefillArgs& a, cudaStream_t s) {
   if (a.k <= 32)
     return m ? gather_mma_as<D, 1, true>(a, grid, smem, s)
              : gather_mma_as<D, 1, false>(a, grid, smem, s);
-  return m ? gather_mma_as<D, 2, true>(a, grid, smem, s)
-           : gather_mma_as<D, 2, false>(a, grid, smem, s);
+  if (a.k <= 64)
+    return m ? gather_mma_as<D, 2, true>(a, grid, smem, s)
+             : gather_mma_as<D, 2, false>(a, grid, smem, s);
+  return m ? gather_mma_as<D, 4, true>(a, grid, smem, s)
+           : gather_mma_as<D, 4, false>(a, grid, smem, s);
 }
 
 }  // namespace

@@ -8,7 +8,7 @@
 namespace ca {
 
 // Largest Top-k the prefill selector holds per row (shared-memory heap).
-constexpr int kPrefillMaxK = 64;
+constexpr int kPrefillMaxK = 128;
 
 struct PrefillArgs {
   const void* Q;   // [B, Hq, nq, d]

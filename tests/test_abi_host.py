@@ -184,7 +184,7 @@ def test_shard_combine_arguments(lib):
 
 
 def test_k_limits(lib):
-    assert _prefill(lib, k=65, C_max=1 + 64 + 65) == binding.CA_ERR_UNSUPPORTED
+    assert _prefill(lib, k=129, C_max=1 + 64 + 129) == binding.CA_ERR_UNSUPPORTED
     assert _decode(lib, k=1025, C_max=1000) == binding.CA_ERR_UNSUPPORTED
 
 

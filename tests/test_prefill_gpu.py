@@ -43,6 +43,20 @@ def test_prefill_edges(dtype, d, n, W, k):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n,W,k", [(2048, 256, 128), (700, 64, 100),
+                                   (130, 1, 128)])
+def test_prefill_k_up_to_128(dtype, d, n, W, k):
+    # the largest prefill Top-k (the 1M decode config's k = 128): most rows
+    # hold more candidates than the tensor-core selector's segments and take
+    # the exact fallback, which the check includes
+    w = workloads.get("prefill_gpt2s_8k").scaled(
+        dtype=dtype, d=d, n=n, W=W, k=k, B=1, Hq=2, Hkv=1, needles=4,
+        needle_gap=128)
+    print(check_prefill(w, workloads.generate(w)))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_prefill_gqa_groups(dtype):
     w = workloads.get("prefill_gpt2s_8k").scaled(
         dtype=dtype, n=700, B=1, Hq=8, Hkv=1, needles=4)
