@@ -24,16 +24,18 @@
 //              key tile), reading the accumulators with tcgen05.ld 32x32b:
 //     pass 1   64 slot maxima per thread (its 32 columns of the even and of the
 //              odd key tiles), rounded toward zero to bf16 and kept in pairs:
-//              256 slots per row.  The k-th largest slot L bounds the row's
-//              k-th best score from below (the top k slots are k distinct
-//              candidates >= L; a negative slot is first moved one bf16 step
-//              down, since rounding toward zero raised it).
+//              256 slots per row; with k <= 32, 32 slots per thread (column
+//              pairs, a three-input fp32 max per two scores): 128 per row.
+//              The k-th largest slot L bounds the row's k-th best score from
+//              below (the top k slots are k distinct candidates >= L; a
+//              negative slot is first moved one bf16 step down, since
+//              rounding toward zero raised it).
 //     pass 2   every candidate >= L is appended to the thread's segment as an
 //              8-byte entry {fp32 score bits, key position} by one predicated
-//              vector store (about 1.1 k entries per row on random data).  A
-//              segment that cannot take 16 more entries moves to one of 16
-//              spare segments; with none left the row goes to the exact
-//              CUDA-core fallback.
+//              vector store (about 1.1 k entries per row on random data),
+//              with a room check every 8 columns.  A segment without room
+//              moves to one of 16 spare segments; with none left the row goes
+//              to the exact CUDA-core fallback.
 //     cut      four lanes per row (one per chunk group) find the exact k-th
 //              best key by bisection on the score bits (and on the positions
 //              only when equal scores straddle it) and write the row's Top-k.
@@ -260,7 +262,11 @@ __device__ __forceinline__ void quad_cut(const unsigned char* seg, int col_own,
   }
 }
 
-template <int D, bool MASS>
+// PAIR: one slot per two columns (128 per row; a three-input max per two
+// scores in pass 1 and half the bound's counting) when k <= 32, where the
+// extra collisions of the best keys in a slot cost a few candidates per row;
+// else one slot per column and tile parity (256 per row).
+template <int D, bool MASS, bool PAIR>
 __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
 prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
                       int P, int maps3d) {
@@ -463,17 +469,34 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
     };
 
     // ---- pass 1: bf16 slot maxima, even tiles in sl[0], odd tiles in sl[1]
+    // (PAIR: fp32 maxima of column pairs over all tiles, in fl)
     uint32_t sl[2][16];
+    float fl[2][16];
 #pragma unroll
     for (int p = 0; p < 2; ++p)
 #pragma unroll
-      for (int x = 0; x < 16; ++x) sl[p][x] = 0xFF80FF80u;  // (-inf, -inf)
-    auto slot_max = [&](const uint32_t (&raw)[32], uint32_t (&s)[16]) {
+      for (int x = 0; x < 16; ++x) {
+        sl[p][x] = 0xFF80FF80u;  // (-inf, -inf)
+        fl[p][x] = -INFINITY;
+      }
+    auto slot_max = [&](const uint32_t (&raw)[32], int p) {
+      if constexpr (PAIR) {
 #pragma unroll
-      for (int x = 0; x < 16; ++x)
-        s[x] = sm100::max_bf16x2(
-            s[x], sm100::cvt_rz_bf16x2(__uint_as_float(raw[2 * x + 1]),
-                                       __uint_as_float(raw[2 * x])));
+        for (int x = 0; x < 16; ++x) {
+          float m3;
+          asm("max.f32 %0, %1, %2, %3;"
+              : "=f"(m3)
+              : "f"(fl[p][x]), "f"(__uint_as_float(raw[2 * x])),
+                "f"(__uint_as_float(raw[2 * x + 1])));
+          fl[p][x] = m3;
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          sl[p][x] = sm100::max_bf16x2(
+              sl[p][x], sm100::cvt_rz_bf16x2(__uint_as_float(raw[2 * x + 1]),
+                                             __uint_as_float(raw[2 * x])));
+      }
     };
     bool live_pass = true;
 #pragma unroll 1
@@ -483,13 +506,13 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
         live_pass = false;
         break;
       }
-      slot_max(raw, sl[0]);
+      slot_max(raw, 0);
       if (t + 1 < T) {
         if (!fetch(t + 1, t + 1, raw)) {
           live_pass = false;
           break;
         }
-        slot_max(raw, sl[1]);
+        slot_max(raw, 1);
       }
     }
     // ---- the slot table: row r's 512 bytes, 16-byte pieces XOR-swizzled
@@ -497,11 +520,27 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
     // over the banks
     {
       uint4* table = reinterpret_cast<uint4*>(seg);
+      if constexpr (PAIR) {
+        // 32 slots, rounded toward zero to bf16, two per word: row r's 256
+        // bytes, 16-byte pieces swizzled by the row
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int piece = (grp * 8 + c) ^ (r & 31);
-        const uint32_t* src = &sl[c >> 2][(c & 3) * 4];
-        table[r * 32 + piece] = make_uint4(src[0], src[1], src[2], src[3]);
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            sl[p][x] = sm100::cvt_rz_bf16x2(fl[p][2 * x + 1], fl[p][2 * x]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int piece = (grp * 4 + c) ^ (r & 15);
+          const uint32_t* src = &sl[c >> 1][(c & 1) * 4];
+          table[r * 16 + piece] = make_uint4(src[0], src[1], src[2], src[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int piece = (grp * 8 + c) ^ (r & 31);
+          const uint32_t* src = &sl[c >> 2][(c & 3) * 4];
+          table[r * 32 + piece] = make_uint4(src[0], src[1], src[2], src[3]);
+        }
       }
     }
     SelBar::sync();
@@ -513,11 +552,14 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
       const uint4* table = reinterpret_cast<const uint4*>(seg);
       // ord codes: hw compares the high halves as is, lw the low halves
       // moved up (a 16-bit code c is compared as c << 16)
-      uint32_t hw[32], lw[32];
+      constexpr int NWD = PAIR ? 16 : 32;  // slot words per lane
+      uint32_t hw[NWD], lw[NWD];
       uint32_t mx = 0u, mn = 0xFFFFu;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = table[row * 32 + ((part * 8 + c) ^ (row & 31))];
+      for (int c = 0; c < NWD / 4; ++c) {
+        const uint4 v = PAIR
+            ? table[row * 16 + ((part * 4 + c) ^ (row & 15))]
+            : table[row * 32 + ((part * 8 + c) ^ (row & 31))];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -542,7 +584,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
         const uint32_t C = c << 16;
         int m = 0;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) m += (hw[x] >= C) + (lw[x] >= C);
+        for (int x = 0; x < NWD; ++x) m += (hw[x] >= C) + (lw[x] >= C);
         m = quad_sum(m);
         const bool up = !done && bit < nb && m >= k;
         tau = up ? c : tau;
@@ -689,8 +731,11 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t s) {
   if (Lay::bytes(P) > budget || P < kCheck + 8) return cudaErrorNotSupported;
   const size_t smem = Lay::bytes(P);
   const bool mass = a.mass != nullptr || a.lse != nullptr;
-  auto kern = mass ? prefill_score_topk_tc<D, true>
-                   : prefill_score_topk_tc<D, false>;
+  const bool pair = a.k <= 32;
+  auto kern = mass ? (pair ? prefill_score_topk_tc<D, true, true>
+                           : prefill_score_topk_tc<D, true, false>)
+                   : (pair ? prefill_score_topk_tc<D, false, true>
+                           : prefill_score_topk_tc<D, false, false>);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.nq + kBM - 1) / kBM, a.Hq, a.B);
