@@ -689,8 +689,16 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
       }
       const uint32_t lob = ord_f32(sh.L[row]);
       uint64_t* out = a.topk + grow * a.k;
+      // entries per lane sized by the warp's fullest lane: the bisection
+      // counts every slot of the array at each step
       if (__all_sync(0xFFFFFFFFu, !live || n_part <= 16))
         quad_cut<16>(seg, cown, n_own, col_x, n_part, live, lob, k, a.k, out,
+                     part);
+      else if (__all_sync(0xFFFFFFFFu, !live || n_part <= 24))
+        quad_cut<24>(seg, cown, n_own, col_x, n_part, live, lob, k, a.k, out,
+                     part);
+      else if (__all_sync(0xFFFFFFFFu, !live || n_part <= 32))
+        quad_cut<32>(seg, cown, n_own, col_x, n_part, live, lob, k, a.k, out,
                      part);
       else
         quad_cut<kCutNE>(seg, cown, n_own, col_x, n_part, live, lob, k, a.k,
