@@ -98,6 +98,21 @@ def test_prefill_adaptive_32k_sampled():
 
 
 @pytest.mark.parametrize("d", [64, 128])
+def test_prefill_beyond_262144(d):
+    """A sequence longer than 2^18 positions (positions are 32-bit in the
+    selector's entries): 600 sampled rows, spread over the length, plus every
+    row sent to the exact fallback."""
+    w = workloads.get("prefill_gpt2s_8k").scaled(
+        d=d, n=300000, B=1, Hq=1, Hkv=1, W=64, k=32, needles=8)
+    x = workloads.generate(w)
+    sel = _sample_rows(w, 600, 7)
+    sel = np.unique(np.concatenate(
+        [sel, np.array([[0, 0, i] for i in (262143, 262144, 262145, 299999)],
+                       dtype=np.int64)]), axis=0)
+    print(check_prefill(w, x, sel=sel, with_fallback_rows=True))
+
+
+@pytest.mark.parametrize("d", [64, 128])
 def test_prefill_equal_keys_take_the_fallback(d):
     """All keys equal: every candidate ties at the pass-1 bound, so rows with
     more candidates than the row buffer holds go through the exact fallback;
