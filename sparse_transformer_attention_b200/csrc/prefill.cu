@@ -970,8 +970,12 @@ bool want_mass(const PrefillArgs& a) {
 template <int D>
 cudaError_t launch_overflow_d(const PrefillArgs& a, cudaStream_t s) {
   const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
+  // A listed row is one CTA's job, latency-bound on its key-row loads: four
+  // CTAs per SM keep more rows in flight (the row count is only known on the
+  // device; CTAs without a row leave at once).
   prof_before(s, "prefill_overflow_rows");
-  prefill_overflow_rows<__nv_bfloat16, D><<<sm_count(), kFbThreads, fb_smem, s>>>(a);
+  prefill_overflow_rows<__nv_bfloat16, D>
+      <<<4 * sm_count(), kFbThreads, fb_smem, s>>>(a);
   prof_after(s);
   return cudaGetLastError();
 }
