@@ -501,6 +501,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 decode_merge_attend(DecodeArgs a) {
   constexpr int DL = D / 32;  // head dims per lane in the gathers
   constexpr int NW = kMergeThreads / 32;
+  static_assert(NW <= 32, "one lane per warp in the final combine");
   constexpr int UG = 4;       // rows in flight per warp
   extern __shared__ __align__(128) unsigned char smem[];
   const int k = a.k;
@@ -889,6 +890,23 @@ decode_merge_attend(DecodeArgs a) {
   __syncthreads();
   const int got = s_m < m ? s_m : m;
   if (m > 0 && s_m != m && tid == 0) raise_flag(a.status, kErrInternal);
+  // idx: C_i = {0} U sorted Top-k U [lo, i], ascending, -1 padded, and |C_i|
+  auto write_idx = [&]() {
+    int32_t* idx_row = a.idx + ((size_t)b * a.Hq + h) * a.C_max;
+    if (count > a.C_max && tid == 0) raise_flag(a.status, kErrCmax);
+    const int64_t wcount = count < a.C_max ? count : a.C_max;
+    for (int64_t r = tid; r < a.C_max; r += kMergeThreads) {
+      int32_t v;
+      if (r >= wcount) v = -1;
+      else if (r < anc) v = 0;
+      else if (r < anc + m) v = (r - anc < got) ? (int32_t)topj[r - anc] : 0;
+      else v = (int32_t)(lo + (r - anc - m));
+      idx_row[r] = v;
+    }
+    if (tid == 0) a.idx_count[(size_t)b * a.Hq + h] = (int32_t)count;
+  };
+  // (k <= 128: topj is sorted already, so the writes overlap the gathers)
+  if (a.kpow2 <= 128) write_idx();
   // Top-k rows, spread over all warps: the score travels with the key, so
   // only V is read (of the rows in this cache)
 #pragma unroll 1
@@ -917,19 +935,27 @@ decode_merge_attend(DecodeArgs a) {
   for (int e = 0; e < DL; ++e) s_ow[warp][lane * DL + e] = acc.o[e];
   __syncthreads();  // every warp is done reading topj
   // C_i = {0} U sorted Top-k U [lo, i], ascending, for the idx output
-  // (the two-level selection wrote it sorted already)
+  // (the k <= 128 path wrote it sorted already)
   if (warp == 0 && a.kpow2 > 128) warp_sort_prefix(topj, got, a.kpow2, lane);
   if (tid >= 32 && tid < 32 + D) {
+    // lane w < NW of each combining warp holds warp w's scale 2^(m_w - M)
+    // (0 for a warp that saw no row)
     const int dd = tid - 32;
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_mw[w]);
-    float l = 0.f, o = 0.f;
-    for (int w = 0; w < NW; ++w) {
-      if (s_lw[w] == 0.f) continue;
-      const float c = exp2f(s_mw[w] - M);
-      l += s_lw[w] * c;
-      o += s_ow[w][dd] * c;
-    }
+    const float mw = lane < NW ? s_mw[lane] : -INFINITY;
+    const float lw = lane < NW ? s_lw[lane] : 0.f;
+    float M = mw;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+    const float cw = lw != 0.f ? exp2f(mw - M) : 0.f;
+    float l = lw * cw;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      o = fmaf(s_ow[w][dd], __shfl_sync(0xFFFFFFFFu, cw, w), o);
     if (shard_part) {
       // this shard's softmax state over its part of C_i: (max, sum, o) in
       // the log2 domain, o not yet divided by the sum (max = -inf, sum = 0
@@ -957,20 +983,11 @@ decode_merge_attend(DecodeArgs a) {
     mass_report(a.mass, a.lse, (size_t)b * a.Hq + h, c.m, c.l, wa.m, wa.l,
                 cand.m, cand.l, s_s0, anc != 0);
   }
-  // the radix path's sorted Top-k must be visible to every thread
-  if (a.kpow2 > 128) __syncthreads();
-  int32_t* idx_row = a.idx + ((size_t)b * a.Hq + h) * a.C_max;
-  if (count > a.C_max && tid == 0) raise_flag(a.status, kErrCmax);
-  const int64_t wcount = count < a.C_max ? count : a.C_max;
-  for (int64_t r = tid; r < a.C_max; r += kMergeThreads) {
-    int32_t v;
-    if (r >= wcount) v = -1;
-    else if (r < anc) v = 0;
-    else if (r < anc + m) v = (r - anc < got) ? (int32_t)topj[r - anc] : 0;
-    else v = (int32_t)(lo + (r - anc - m));
-    idx_row[r] = v;
+  // the radix path's Top-k, sorted by warp 0 above, once every thread sees it
+  if (a.kpow2 > 128) {
+    __syncthreads();
+    write_idx();
   }
-  if (tid == 0) a.idx_count[(size_t)b * a.Hq + h] = (int32_t)count;
 }
 
 
