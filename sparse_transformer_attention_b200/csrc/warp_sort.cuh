@@ -29,29 +29,6 @@ __device__ __forceinline__ void warp_bitonic(uint32_t (&v)[NPL], int lane) {
   }
 }
 
-// The same network on 64-bit values.
-template <int NPL>
-__device__ __forceinline__ void warp_bitonic64(uint64_t (&v)[NPL], int lane) {
-#pragma unroll
-  for (int size = 2; size <= 32 * NPL; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      uint64_t nv[NPL];
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) {
-        const int e = t * 32 + lane;
-        const uint64_t other = (stride >= 32)
-            ? v[t ^ (stride >> 5)]
-            : __shfl_xor_sync(0xFFFFFFFFu, v[t], stride);
-        const bool up = (e & size) == 0, lower = (e & stride) == 0;
-        nv[t] = (lower == up) ? min(v[t], other) : max(v[t], other);
-      }
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) v[t] = nv[t];
-    }
-  }
-}
-
 template <int NPL>
 __device__ __forceinline__ void warp_sort_n(uint32_t* a, int n, int lane) {
   uint32_t v[NPL];
