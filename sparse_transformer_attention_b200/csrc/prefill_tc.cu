@@ -5,20 +5,23 @@
 //
 // One CTA per 128-query tile of one (batch, head):
 //   TMA warps  the key tiles 0..T-1 twice (two passes)
-//              through a ring of 32 KB stages, one stage per producer warp
-//              (three at d = 64, two at d = 128: warps 0, 2 and 3).  Every
-//              copy moves 32 KB (two 128-key tiles at d = 64, one tile with
-//              both 64-column halves at d = 128).  On this part the copy rate
-//              per SM grows with the size of each copy and with the number of
-//              threads issuing them (one thread's copies do not overlap: 16 KB
-//              copies from one thread stream at about a quarter of what 32 KB
-//              copies from two threads do).  At d = 64 a copy outlasts the MMAs
-//              of its two tiles, hence the third stage.
+//              through a ring of two 32 KB stages, one stage per producer
+//              warp (warps 0 and 2).  Every copy moves 32 KB (two 128-key
+//              tiles at d = 64, one tile with both 64-column halves at
+//              d = 128).  On this part the copy rate per SM grows with the
+//              size of each copy and with the number of threads issuing them
+//              (one thread's copies do not overlap: 16 KB copies from one
+//              thread stream at about a quarter of what 32 KB copies from two
+//              threads do).
 //   warp 1     MMA: tcgen05.mma kind::f16, M = N = 128, bf16 in, fp32 out, into
-//              three 128-column TMEM accumulators.  A (the Q tile) is read
-//              from TMEM, where the first selector warps store it once (their
-//              rows, straight from global memory): that leaves its 16-32 KB of
-//              shared memory to the candidate segments.
+//              128-column TMEM accumulators.  At d = 64 the Q tile (A) sits in
+//              shared memory, written once by the first selector warps in the
+//              128-byte swizzle, and TMEM holds four accumulators; at d = 128
+//              Q is read from TMEM (64 columns after three accumulators), which
+//              leaves its 32 KB of shared memory to the candidate segments.
+//              Pass 1 is bound by the round trip of an accumulator (MMA,
+//              commit, every selector warp's read and release), so the count
+//              of accumulators sets its pace.
 //   16 warps   selectors (after the TMA and MMA warps), thread = (query row,
 //              32-column chunk group of every
 //              key tile), reading the accumulators with tcgen05.ld 32x32b:
@@ -60,8 +63,7 @@ constexpr int kBM = kPrefillTileRows;  // query rows per CTA
 constexpr int kBN = 128;               // keys per accumulator tile
 constexpr int kSelWarps = 16;          // 4 chunk groups x 4 TMEM lane quarters
 constexpr int kSelThreads = 32 * kSelWarps;
-constexpr int kTmemBufs = 3;
-constexpr int kQCol = kTmemBufs * 128;  // TMEM columns of the Q tile
+constexpr int kTmemBufs = 4;  // most accumulators (d = 64; three at 128)
 constexpr uint32_t kStageBytes = 32768;
 constexpr uint32_t kBlockBytes = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kPool = 16;                    // spare segments per CTA
@@ -78,12 +80,19 @@ using SelBar = GroupBarrier<1, kSelThreads>;
 template <int D>
 struct Layout {
   static constexpr int KT = D == 64 ? 2 : 1;  // key tiles per stage
-  static constexpr int kStages = D == 64 ? 3 : 2;  // = producer warps
-  // warp 0 and warps 2.. produce, warp 1 issues MMAs, then the selectors
+  static constexpr int kStages = 2;  // = producer warps
+  // At d = 64 the Q tile (16 KB) sits in shared memory and TMEM holds four
+  // 128-column accumulators; at d = 128 Q (64 TMEM columns) sits in TMEM
+  // after three accumulators, and its 32 KB stay with the segments.
+  static constexpr bool kQSmem = D == 64;
+  static constexpr int kBufs = kQSmem ? 4 : 3;
+  static constexpr int kQCol = 3 * 128;  // TMEM columns of Q at d = 128
+  // warp 0 and warp 2 produce, warp 1 issues MMAs, then the selectors
   static constexpr int kFirstSel = kStages + 1;
   static constexpr int kThreads = 32 * kFirstSel + kSelThreads;
   static constexpr size_t k_off = 0;
-  static constexpr size_t seg_off = k_off + (size_t)kStages * kStageBytes;
+  static constexpr size_t q_off = k_off + (size_t)kStages * kStageBytes;
+  static constexpr size_t seg_off = q_off + (kQSmem ? (size_t)kBM * 128 : 0);
   // segments, or the pass-1 slot table (128 rows x 256 bf16) before them
   __host__ __device__ static size_t bytes(int P) {
     size_t seg = (size_t)P * kEntStride;
@@ -274,10 +283,13 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
   constexpr int KT = Lay::KT;
   constexpr int kStages = Lay::kStages;
   constexpr int kFirstSel = Lay::kFirstSel;
+  constexpr int kBufs = Lay::kBufs;
+  constexpr int kQCol = Lay::kQCol;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sK = smem + Lay::k_off;
+  unsigned char* sQ = smem + Lay::q_off;  // d = 64: the Q tile, 128-byte rows
   unsigned char* seg = smem + Lay::seg_off;
   __shared__ Shared sh;
 
@@ -296,7 +308,7 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
     }
     sm100::mbar_init(&sh.qfull, 4);  // the four Q-writing selector warps
     sm100::mbar_init(&sh.never, 1);
-    for (int t = 0; t < kTmemBufs; ++t) {
+    for (int t = 0; t < kBufs; ++t) {
       sm100::mbar_init(&sh.tfull[t], 1);
       sm100::mbar_init(&sh.tempty[t], kSelWarps);
     }
@@ -378,9 +390,9 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
 #pragma unroll
           for (int q = 0; q < KT; ++q) {
             if (t0 + q >= T) break;
-            const int buf = tt % kTmemBufs;
-            if (tt >= kTmemBufs &&
-                !sm100::wait_or_abort(&sh.tempty[buf], ((tt / kTmemBufs) & 1) ^ 1,
+            const int buf = tt % kBufs;
+            if (tt >= kBufs &&
+                !sm100::wait_or_abort(&sh.tempty[buf], ((tt / kBufs) & 1) ^ 1,
                                       abort_flag, a.status, a.wait_ns)) {
               ok = false;
               break;
@@ -391,9 +403,16 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-              sm100::mma_bf16_ts(d_tmem, tmem + kQCol + kk * 8,
-                                 sm100::desc_k_sw128(kt + off), idesc,
-                                 kk > 0 ? 1u : 0u);
+              if constexpr (Lay::kQSmem)
+                sm100::mma_bf16(d_tmem,
+                                sm100::desc_k_sw128(sm100::smem_u32(sQ) +
+                                                    (kk & 3) * 32),
+                                sm100::desc_k_sw128(kt + off), idesc,
+                                kk > 0 ? 1u : 0u);
+              else
+                sm100::mma_bf16_ts(d_tmem, tmem + kQCol + kk * 8,
+                                   sm100::desc_k_sw128(kt + off), idesc,
+                                   kk > 0 ? 1u : 0u);
             }
             sm100::mma_commit(&sh.tfull[buf]);
             ++tt;
@@ -403,8 +422,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
       }
       // The last commit covers every MMA issued: wait for it before exit.
       if (tt > 0 &&
-          !sm100::mbar_wait(&sh.tfull[(tt - 1) % kTmemBufs],
-                            ((tt - 1) / kTmemBufs) & 1, kDrainWaitNs))
+          !sm100::mbar_wait(&sh.tfull[(tt - 1) % kBufs],
+                            ((tt - 1) / kBufs) & 1, kDrainWaitNs))
         raise_flag(a.status, kErrTimeout);
     }
   } else {
@@ -417,7 +436,25 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
     const int hi = sh.hi[r];
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + grp * 32;
 
-    if (grp == 0) {
+    if (grp == 0 && Lay::kQSmem) {
+      // the Q tile into shared memory: this warp's 32 rows, each thread its
+      // own 128-byte row, 16-byte pieces placed as the 128-byte swizzle
+      // places them (piece c of row r at c ^ (r % 8)), zeros past the last
+      // query row; then made visible to the tensor core's reads
+      const bool qv = i0 + r < a.nq;
+      const uint4* qp = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(a.Q) +
+          ((size_t)(b * a.Hq + h) * a.nq + (qv ? i0 + r : 0)) * D);
+      uint4 v[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[c] = qv ? qp[c] : make_uint4(0u, 0u, 0u, 0u);
+      uint4* qrow = reinterpret_cast<uint4*>(sQ + (size_t)r * 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) qrow[c ^ (r & 7)] = v[c];
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sh.qfull);
+    } else if (grp == 0) {
       // the Q tile into TMEM columns kQCol..: this warp's 32 rows, each
       // thread its own row as bf16 pairs (zeros past the last query row)
       const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16) + kQCol;
@@ -448,9 +485,9 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
     // thread's row and chunk, non-candidates (j = 0, the window, the future)
     // replaced by NaN.
     auto fetch = [&](int tt, int t, uint32_t (&raw)[32]) -> bool {
-      const int buf = tt % kTmemBufs;
+      const int buf = tt % kBufs;
       if (!__all_sync(0xFFFFFFFFu,
-                      sm100::wait_or_abort(&sh.tfull[buf], (tt / kTmemBufs) & 1,
+                      sm100::wait_or_abort(&sh.tfull[buf], (tt / kBufs) & 1,
                                            abort_flag, a.status, a.wait_ns)))
         return false;
       sm100::tc_fence_after();
