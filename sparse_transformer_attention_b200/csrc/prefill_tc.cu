@@ -367,24 +367,32 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
       if (!drained) raise_flag(a.status, kErrTimeout);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0 && T > 0) {
+    // ---------------- MMA issuer: the whole warp runs the loop (waits,
+    // addresses and descriptors warp-uniform); one elected lane issues each
+    // MMA and commit
+    if (T > 0) {
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kBN);
       const uint32_t ak = sm100::smem_u32(sK);
+      const bool leader = sm100::elect_one();
       int tt = 0;  // accumulator tiles issued, both passes
       if (a.stall_ns) {
         // Failure-path test hook: wait on a barrier that nothing signals, so
         // the wait runs out, raises the time-out flag and aborts every wait
         // of the CTA; the kernel then leaves through its normal path.
-        sm100::wait_or_abort(&sh.never, 0, abort_flag, a.status, a.stall_ns);
+        if (leader)
+          sm100::wait_or_abort(&sh.never, 0, abort_flag, a.status, a.stall_ns);
+        __syncwarp();
       }
-      if (sm100::wait_or_abort(&sh.qfull, 0, abort_flag, a.status, a.wait_ns)) {
+      if (__all_sync(0xFFFFFFFFu,
+                     sm100::wait_or_abort(&sh.qfull, 0, abort_flag, a.status,
+                                          a.wait_ns))) {
         bool ok = true;
         for (int u = 0; u < 2 * TS && ok; ++u) {
           const int s = u % kStages;
           const uint32_t ph = (u / kStages) & 1;
-          if (!sm100::wait_or_abort(&sh.kfull[s], ph, abort_flag, a.status,
-                                    a.wait_ns))
+          if (!__all_sync(0xFFFFFFFFu,
+                          sm100::wait_or_abort(&sh.kfull[s], ph, abort_flag,
+                                               a.status, a.wait_ns)))
             break;
           const int t0 = (u < TS ? u : u - TS) * KT;
 #pragma unroll
@@ -392,36 +400,43 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
             if (t0 + q >= T) break;
             const int buf = tt % kBufs;
             if (tt >= kBufs &&
-                !sm100::wait_or_abort(&sh.tempty[buf], ((tt / kBufs) & 1) ^ 1,
-                                      abort_flag, a.status, a.wait_ns)) {
+                !__all_sync(0xFFFFFFFFu,
+                            sm100::wait_or_abort(&sh.tempty[buf],
+                                                 ((tt / kBufs) & 1) ^ 1,
+                                                 abort_flag, a.status,
+                                                 a.wait_ns))) {
               ok = false;
               break;
             }
             sm100::tc_fence_after();
             const uint32_t d_tmem = tmem + buf * kBN;
             const uint32_t kt = ak + s * kStageBytes + q * kBlockBytes;
+            if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-              if constexpr (Lay::kQSmem)
-                sm100::mma_bf16(d_tmem,
-                                sm100::desc_k_sw128(sm100::smem_u32(sQ) +
-                                                    (kk & 3) * 32),
-                                sm100::desc_k_sw128(kt + off), idesc,
-                                kk > 0 ? 1u : 0u);
-              else
-                sm100::mma_bf16_ts(d_tmem, tmem + kQCol + kk * 8,
-                                   sm100::desc_k_sw128(kt + off), idesc,
-                                   kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+                if constexpr (Lay::kQSmem)
+                  sm100::mma_bf16(d_tmem,
+                                  sm100::desc_k_sw128(sm100::smem_u32(sQ) +
+                                                      (kk & 3) * 32),
+                                  sm100::desc_k_sw128(kt + off), idesc,
+                                  kk > 0 ? 1u : 0u);
+                else
+                  sm100::mma_bf16_ts(d_tmem, tmem + kQCol + kk * 8,
+                                     sm100::desc_k_sw128(kt + off), idesc,
+                                     kk > 0 ? 1u : 0u);
+              }
+              sm100::mma_commit(&sh.tfull[buf]);
             }
-            sm100::mma_commit(&sh.tfull[buf]);
+            __syncwarp();
             ++tt;
           }
-          sm100::mma_commit(&sh.kempty[s]);
+          if (leader) sm100::mma_commit(&sh.kempty[s]);
+          __syncwarp();
         }
       }
       // The last commit covers every MMA issued: wait for it before exit.
-      if (tt > 0 &&
+      if (leader && tt > 0 &&
           !sm100::mbar_wait(&sh.tfull[(tt - 1) % kBufs],
                             ((tt - 1) / kBufs) & 1, kDrainWaitNs))
         raise_flag(a.status, kErrTimeout);

@@ -218,6 +218,18 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
+// One lane of the (converged) warp: true there, false elsewhere.  Issuing an
+// MMA under this predicate inside a warp-uniform loop keeps its operands in
+// uniform registers; a loop run by one lane alone pays a conversion per
+// operand and issues several times slower.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{ .reg .pred P; elect.sync _|P, 0xFFFFFFFF; selp.b32 %0, 1, 0, P; }"
+      : "=r"(p));
+  return p != 0;
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread
 // has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
