@@ -289,19 +289,24 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
       if (!drained) raise_flag(a.status, kErrTimeout);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
+    // ---------------- MMA issuer: the whole warp runs the loop (waits,
+    // addresses and descriptors warp-uniform); one elected lane writes the
+    // tile positions and issues each MMA, commit and arrival
+    {
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kKeys, kN);
       const uint32_t aq = sm100::smem_u32(sQ);
       const uint32_t ak = sm100::smem_u32(sK);
+      const bool leader = sm100::elect_one();
       int tt = 0, real = 0;
       bool ok = true;
       // the next accumulator buffer, once the selectors have released it
       auto take_buf = [&]() -> int {
         const int tb = tt & (kTBufs - 1);
         if (tt >= kTBufs &&
-            !sm100::wait_or_abort(&sh->tempty[tb], ((tt / kTBufs) & 1) ^ 1,
-                                  abort_flag, a.status, a.wait_ns))
+            !__all_sync(0xFFFFFFFFu,
+                        sm100::wait_or_abort(&sh->tempty[tb],
+                                             ((tt / kTBufs) & 1) ^ 1,
+                                             abort_flag, a.status, a.wait_ns)))
           return -1;
         return tb;
       };
@@ -309,14 +314,20 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
         // Failure-path test hook: wait on a barrier that nothing signals, so
         // the wait runs out, raises the time-out flag and aborts every wait
         // of the CTA; the kernel then leaves through its normal path.
-        sm100::wait_or_abort(&sh->never, 0, abort_flag, a.status, a.stall_ns);
+        if (leader)
+          sm100::wait_or_abort(&sh->never, 0, abort_flag, a.status,
+                               a.stall_ns);
+        __syncwarp();
       }
-      if (sm100::wait_or_abort(&sh->qfull, 0, abort_flag, a.status,
-                               a.wait_ns)) {
+      if (__all_sync(0xFFFFFFFFu,
+                     sm100::wait_or_abort(&sh->qfull, 0, abort_flag, a.status,
+                                          a.wait_ns))) {
         for (int u = 0; ok; ++u) {
           const int s = u % NS;
-          if (!sm100::wait_or_abort(&sh->full[s], (u / NS) & 1, abort_flag,
-                                    a.status, a.wait_ns))
+          if (!__all_sync(0xFFFFFFFFu,
+                          sm100::wait_or_abort(&sh->full[s], (u / NS) & 1,
+                                               abort_flag, a.status,
+                                               a.wait_ns)))
             break;
           const int pos = *(volatile int*)&sh->spos[s];
           if (pos < 0) {
@@ -328,9 +339,12 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
                 ok = false;
                 break;
               }
-              sh->tpos[tb] = -1;
-              sm100::mbar_arrive(&sh->tfull[tb]);
-              sm100::mbar_arrive(&sh->tfull[tb]);
+              if (leader) {
+                sh->tpos[tb] = -1;
+                sm100::mbar_arrive(&sh->tfull[tb]);
+                sm100::mbar_arrive(&sh->tfull[tb]);
+              }
+              __syncwarp();
               ++tt;
             }
             break;
@@ -342,27 +356,31 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
               ok = false;
               break;
             }
-            sh->tpos[tb] = pos + q * kKeys;
             sm100::tc_fence_after();
             const uint32_t kt = ak + s * kStage + q * 16384;
+            if (leader) {
+              sh->tpos[tb] = pos + q * kKeys;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t offk = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t offq = (kk >> 2) * (kN * 128) + (kk & 3) * 32;
-              sm100::mma_bf16(tmem + tb * kN, sm100::desc_k_sw128(kt + offk),
-                              sm100::desc_k_sw128(aq + offq), idesc,
-                              kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t offk = (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint32_t offq = (kk >> 2) * (kN * 128) + (kk & 3) * 32;
+                sm100::mma_bf16(tmem + tb * kN, sm100::desc_k_sw128(kt + offk),
+                                sm100::desc_k_sw128(aq + offq), idesc,
+                                kk > 0 ? 1u : 0u);
+              }
+              sm100::mma_commit(&sh->tfull[tb]);
+              sm100::mbar_arrive(&sh->tfull[tb]);  // releases the tpos write
             }
-            sm100::mma_commit(&sh->tfull[tb]);
-            sm100::mbar_arrive(&sh->tfull[tb]);  // releases the tpos write
+            __syncwarp();
             ++tt;
             real = tt;
           }
-          sm100::mma_commit(&sh->empty[s]);
+          if (leader) sm100::mma_commit(&sh->empty[s]);
+          __syncwarp();
         }
       }
       // The last commit covers every MMA issued: wait for it before exit.
-      if (real > 0 &&
+      if (leader && real > 0 &&
           !sm100::mbar_wait(&sh->tfull[(real - 1) & (kTBufs - 1)],
                             ((real - 1) / kTBufs) & 1, kDrainWaitNs))
         raise_flag(a.status, kErrTimeout);
