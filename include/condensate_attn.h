@@ -55,6 +55,13 @@
  * set flags in the workspace's status word; condensate_attn_status() waits
  * for the stream and reports them.  The status word is cleared at the start
  * of every call that uses the workspace.  Inputs must be finite.
+ *
+ * Debug build: `python -m sparse_transformer_attention_b200.build --debug`
+ * compiles the same sources with CA_DEBUG into libcondensate_attn_debug.so
+ * (same entry points).  Its kernels also check the indexes that the release
+ * build keeps in range by construction (shared-memory segment cursors, list
+ * slots, survivor slots, rows listed for the exact fallback); a failed check
+ * skips the access and raises CA_ERR_BOUNDS instead of a memory fault.
  */
 #ifndef CONDENSATE_ATTN_H
 #define CONDENSATE_ATTN_H
@@ -81,8 +88,10 @@ typedef enum {
   CA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed            */
   CA_ERR_TIMEOUT = 6,     /* a bounded device wait gave up (status query)    */
   CA_ERR_DEVICE_ARG = 7,  /* W_i out of range or set overflowing C_max      */
-  CA_ERR_INTERNAL = 8     /* an internal check failed on the device: the
+  CA_ERR_INTERNAL = 8,    /* an internal check failed on the device: the
                              results of that call are invalid (a bug)      */
+  CA_ERR_BOUNDS = 9       /* debug build only: an index check failed on the
+                             device and the access was skipped (a bug)     */
 } ca_status;
 
 typedef enum { CA_F32 = 0, CA_BF16 = 1 } ca_dtype;
@@ -291,7 +300,8 @@ CA_API ca_status condensate_attn_decode_noalloc_status(void* stream);
 
 /*
  * Waits for `stream`, then reads and clears the device status word of
- * `workspace`.  The kernels raise four flags there:
+ * `workspace`.  The kernels raise four flags there (five in the debug
+ * build):
  *   W_i below 1                      -> CA_ERR_DEVICE_ARG (the row is run
  *                                       with a window of 1)
  *   |C_i| larger than C_max          -> CA_ERR_DEVICE_ARG (idx holds the
@@ -299,7 +309,10 @@ CA_API ca_status condensate_attn_decode_noalloc_status(void* stream);
  *                                       true size)
  *   a bounded device wait ran out    -> CA_ERR_TIMEOUT (outputs invalid)
  *   an internal check failed         -> CA_ERR_INTERNAL (outputs invalid)
- * The time-out outranks the argument flags, which outrank the internal one.
+ *   (debug build) an index check     -> CA_ERR_BOUNDS (outputs invalid)
+ *   failed
+ * The time-out outranks the argument flags, which outrank the internal one,
+ * which outranks the index check.
  * CA_OK when no flag is set; CA_ERR_CUDA if the wait or copy itself failed.
  */
 CA_API ca_status condensate_attn_status(void* workspace, void* stream);
@@ -335,6 +348,11 @@ CA_API int condensate_attn_profile_stop(const char** names, float* ms,
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 CA_API int condensate_attn_version(void);
+
+/* Flags of the loaded build: CA_BUILD_DEBUG when it was compiled with
+ * CA_DEBUG (the index-checking debug build), 0 for the release build. */
+#define CA_BUILD_DEBUG 1
+CA_API int condensate_attn_build_flags(void);
 
 #ifdef __cplusplus
 }

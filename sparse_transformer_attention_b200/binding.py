@@ -15,6 +15,11 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcondensate_attn.so")
+# the CA_DEBUG build (same entry points; kernels that also check the indexes
+# the release build keeps in range by construction, raising CA_ERR_BOUNDS)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libcondensate_attn_debug.so")
+if os.environ.get("CONDENSATE_ATTN_DEBUG") == "1":
+    LIB_PATH = DEBUG_LIB_PATH
 
 CA_OK = 0
 CA_ERR_INVALID_ARG = 1
@@ -25,6 +30,7 @@ CA_ERR_CUDA = 5
 CA_ERR_TIMEOUT = 6
 CA_ERR_DEVICE_ARG = 7
 CA_ERR_INTERNAL = 8
+CA_ERR_BOUNDS = 9
 
 CA_F32 = 0
 CA_BF16 = 1
@@ -76,6 +82,7 @@ SIGNATURES = {
     "condensate_attn_test_stall": (_I, [ctypes.c_ulonglong]),
     "condensate_attn_status_string": (ctypes.c_char_p, [_I]),
     "condensate_attn_version": (_I, []),
+    "condensate_attn_build_flags": (_I, []),
     "condensate_attn_profile_start": (_I, [_I]),
     "condensate_attn_profile_stop": (_I, [ctypes.POINTER(ctypes.c_char_p),
                                           ctypes.POINTER(ctypes.c_float), _I]),
@@ -108,6 +115,20 @@ def load(path: Optional[str] = None):
     if path is None:
         _lib = lib
     return lib
+
+
+def use_library(lib=None):
+    """Make `lib` (a path, a library load() returned, or None for LIB_PATH)
+    the library every call of this module goes through; returns the one
+    used before (None if none was loaded yet)."""
+    global _lib
+    prev = _lib
+    if isinstance(lib, ctypes.CDLL):
+        _lib = lib
+    else:
+        _lib = None
+        _lib = load(lib)
+    return prev
 
 
 def status_string(code: int) -> str:

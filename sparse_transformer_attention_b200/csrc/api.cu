@@ -140,7 +140,15 @@ ca_status launch_status(cudaError_t e) {
 
 extern "C" {
 
-int condensate_attn_version(void) { return 300; }
+int condensate_attn_version(void) { return 301; }
+
+int condensate_attn_build_flags(void) {
+#ifdef CA_DEBUG
+  return CA_BUILD_DEBUG;
+#else
+  return 0;
+#endif
+}
 
 const char* condensate_attn_status_string(ca_status s) {
   switch (s) {
@@ -153,6 +161,7 @@ const char* condensate_attn_status_string(ca_status s) {
     case CA_ERR_TIMEOUT: return "device wait timed out";
     case CA_ERR_DEVICE_ARG: return "device-side argument out of range";
     case CA_ERR_INTERNAL: return "internal consistency check failed on the device";
+    case CA_ERR_BOUNDS: return "index check of the debug build failed on the device";
   }
   return "unknown status";
 }
@@ -387,6 +396,7 @@ ca_status condensate_attn_status(void* workspace, void* stream) {
   if (word & ca::kErrTimeout) return CA_ERR_TIMEOUT;
   if (word & (ca::kErrWindow | ca::kErrCmax)) return CA_ERR_DEVICE_ARG;
   if (word & ca::kErrInternal) return CA_ERR_INTERNAL;
+  if (word & ca::kErrBounds) return CA_ERR_BOUNDS;
   return CA_OK;
 }
 

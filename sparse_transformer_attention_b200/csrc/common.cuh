@@ -12,6 +12,7 @@ constexpr uint32_t kErrWindow = 1u;    // a window below 1 or k_h outside [0, k]
 constexpr uint32_t kErrTimeout = 2u;   // a bounded wait ran out
 constexpr uint32_t kErrCmax = 4u;      // |C_i| larger than C_max
 constexpr uint32_t kErrInternal = 8u;  // internal capacity check failed
+constexpr uint32_t kErrBounds = 16u;   // (debug builds) an index check failed
 
 constexpr int kStatusBytes = 256;      // status area at the workspace start
 
@@ -24,6 +25,27 @@ constexpr uint64_t kDrainWaitNs = 2000000000ull;     // 2 s
 
 __device__ __forceinline__ void raise_flag(uint32_t* status, uint32_t bit) {
   atomicOr(status, bit);
+}
+
+// Index checks of the debug build.  Built with CA_DEBUG, the kernels check
+// the indexes that the release build keeps in range by construction (the
+// cursors of the prefill selector's shared-memory segments, the slots of the
+// decode score pass's per-head lists, the merge's survivor slots, the rows
+// listed for the exact fallback): a failed check raises kErrBounds and the
+// access is skipped, so a bug shows as a status code instead of a memory
+// fault.  The release build compiles every check to `true`.
+#ifdef CA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t* status) {
+  if constexpr (kDebugChecks) {
+    if (!ok) raise_flag(status, kErrBounds);
+    return ok;
+  } else {
+    return true;
+  }
 }
 
 // Order-preserving map of an fp32 score to uint32: a > b (as reals) iff

@@ -727,7 +727,8 @@ decode_merge_attend(DecodeArgs a) {
           const bool keep = key >= F;  // F >= 1: real keys only
           const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
           if (keep) {
-            surv[beg + w + __popc(bal & ((1u << lane) - 1u))] = key;
+            const int slot = beg + w + __popc(bal & ((1u << lane) - 1u));
+            if (in_bounds(slot < end, a.status)) surv[slot] = key;
             if (!select_only) {
               const char* row = reinterpret_cast<const char*>(
                   Vg - lane * DL + row_of(key_index(key)));

@@ -449,13 +449,14 @@ decode_score_topk_tc(const __grid_constant__ CUtensorMap tmQ,
           if (m == 0) {
             // first stretch: every key of the tile goes in at its own slot
             // (a key outside this head's candidates as an empty key)
-            buf[(size_t)h * cap + t * kKeys + kq] =
-                cand ? make_key(sc, (uint32_t)j) : 0ull;
+            if (in_bounds(t * kKeys + kq < cap, a.status))
+              buf[(size_t)h * cap + t * kKeys + kq] =
+                  cand ? make_key(sc, (uint32_t)j) : 0ull;
           } else if (cand && sc >= thr_f[h]) {
             const uint64_t key = make_key(sc, (uint32_t)j);
             if (key > thr[h]) {
               const int p = atomicAdd(&sh->cnt[h], 1);
-              buf[(size_t)h * cap + p] = key;
+              if (in_bounds(p < cap, a.status)) buf[(size_t)h * cap + p] = key;
             }
           }
         }

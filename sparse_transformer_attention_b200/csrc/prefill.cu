@@ -84,9 +84,13 @@ prefill_overflow_rows(PrefillArgs a) {
   __shared__ int s_n, s_kk, s_w;
   __shared__ uint64_t s_T;
   __shared__ SelectState<1> st;
-  const uint32_t nrows = *a.ovf_count;
+  const uint32_t rows = (uint32_t)(a.B * a.Hq * a.nq);
+  uint32_t nrows = *a.ovf_count;
+  // debug builds: the list holds at most one entry per row, each a row
+  if (!in_bounds(nrows <= rows, a.status)) nrows = rows;
   for (uint32_t it = blockIdx.x; it < nrows; it += gridDim.x) {
     const uint32_t grow = a.ovf_rows[it];
+    if (!in_bounds(grow < rows, a.status)) continue;
     const int r = (int)(grow % (uint32_t)a.nq);
     const uint32_t bh = grow / (uint32_t)a.nq;
     const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);

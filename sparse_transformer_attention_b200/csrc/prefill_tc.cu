@@ -683,6 +683,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
           ovf = true;
         }
       }
+      // debug builds: the next run's kCheck entries must fit the segment
+      if (!ovf && !in_bounds(cur <= lim, a.status)) ovf = true;
     };
 #pragma unroll 1
     for (int t = 0; t < T && live_pass; ++t) {
@@ -721,7 +723,12 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
       const int x = sh.xcol[cown];
       const int n_part = n_own + (x >= 0 ? sh.xcnt[cown] : 0);
       const int col_x = kSelThreads + (x >= 0 ? x : 0);
-      const bool bad = quad_sum(sh.ovf[cown] || n_part > kCutNE) > 0;
+      // debug builds: the entry counts must lie within the segments
+      const bool seg_ok = in_bounds(
+          n_own <= P && (x < 0 || (x < kPool && sh.xcnt[cown] <= P)),
+          a.status);
+      const bool bad =
+          quad_sum(sh.ovf[cown] || n_part > kCutNE || !seg_ok) > 0;
       const size_t grow = (size_t)(b * a.Hq + h) * a.nq + rq;
       bool live = rq < a.nq;
       if constexpr (MASS) {
@@ -735,7 +742,8 @@ prefill_score_topk_tc(const __grid_constant__ CUtensorMap tmK, PrefillArgs a,
         // listed for the exact fallback pass, which writes this row
         if (part == 0) {
           const uint32_t pos = atomicAdd(a.ovf_count, 1u);
-          a.ovf_rows[pos] = (uint32_t)grow;
+          if (in_bounds(pos < (uint32_t)(a.B * a.Hq * a.nq), a.status))
+            a.ovf_rows[pos] = (uint32_t)grow;
         }
         live = false;
       }

@@ -34,7 +34,8 @@ def test_header_lists_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     for name in header_functions():
         assert hasattr(lib, name), name
-    assert lib.condensate_attn_version() == 300
+    assert lib.condensate_attn_version() == 301
+    assert lib.condensate_attn_build_flags() == 0  # the release build
 
 
 def test_status_strings(lib):
