@@ -21,6 +21,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -123,6 +124,14 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text with C/C++ comments and layout removed, so that the hash
+    below follows changes of the code only."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel):
     csrc = os.path.join(ROOT, "sparse_transformer_attention_b200", "csrc")
     own = KERNEL_SOURCES.get(kernel)
@@ -130,7 +139,7 @@ def kernel_source_hash(kernel):
     for fn in sorted(os.listdir(csrc)):
         if fn.endswith(".cuh") or (fn.endswith(".cu") and
                                    (own is None or fn in own)):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+            h.update(_code_only(open(os.path.join(csrc, fn)).read()).encode())
     return h.hexdigest()[:16]
 
 
