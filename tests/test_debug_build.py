@@ -95,3 +95,27 @@ def test_debug_decode_index_checks_clean(debug_calls, dtype, L, W, k, Hq, Hkv):
     w = workloads.get("decode_131k").scaled(
         dtype=dtype, n=L, W=W, k=k, B=2, Hq=Hq, Hkv=Hkv, d=128, needles=16)
     print(check_decode(w, workloads.generate(w)))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["decode_131k", "prefill_gpt2s_8k"])
+def test_debug_build_full_size_matches_release(dlib, name):
+    """The benchmarked workloads at full size through both builds: the debug
+    build's checks stay clean and its results equal the release build's
+    bit for bit (the checks only add branches around accesses)."""
+    import numpy as np
+    import torch
+    from gpu_common import run_decode, run_prefill
+    w = workloads.get(name)
+    x = workloads.generate(w)
+    run = run_decode if w.kind == "decode" else run_prefill
+    as_np = lambda t: t.cpu().numpy() if isinstance(t, torch.Tensor) else t
+    rel = [as_np(t) for t in run(w, x)[:3]]
+    prev = binding.use_library(binding.DEBUG_LIB_PATH)
+    try:
+        assert binding.load().condensate_attn_build_flags() == 1
+        dbg = [as_np(t) for t in run(w, x)[:3]]
+    finally:
+        binding.use_library(prev)
+    for a, b in zip(rel, dbg):
+        assert np.array_equal(a, b)
