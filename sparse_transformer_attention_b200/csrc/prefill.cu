@@ -37,6 +37,24 @@ struct RawRow {
 #pragma unroll
     for (int c = 0; c < kWords; ++c) w[c] = __ldg(s + c);
   }
+  // 16-byte piece c as fp32 (8 bf16 or 4 fp32 elements)
+  __device__ __forceinline__ void piece_f32(int c, float* f) const {
+    if constexpr (sizeof(T) == 2) {
+      f[0] = bf16lo(w[c].x);
+      f[1] = bf16hi(w[c].x);
+      f[2] = bf16lo(w[c].y);
+      f[3] = bf16hi(w[c].y);
+      f[4] = bf16lo(w[c].z);
+      f[5] = bf16hi(w[c].z);
+      f[6] = bf16lo(w[c].w);
+      f[7] = bf16hi(w[c].w);
+    } else {
+      f[0] = __uint_as_float(w[c].x);
+      f[1] = __uint_as_float(w[c].y);
+      f[2] = __uint_as_float(w[c].z);
+      f[3] = __uint_as_float(w[c].w);
+    }
+  }
   __device__ __forceinline__ void to_f32(float (&f)[DL]) const {
     if constexpr (sizeof(T) == 2) {
 #pragma unroll
@@ -69,18 +87,19 @@ struct RawRow {
 // exactly the k keys >= T, so a key below T can never be selected), and the
 // CTA radix select runs only when the buffer could not take another chunk,
 // and once at the end.
-constexpr int kFbThreads = 256;
+constexpr int kFbThreads = 512;
+constexpr int kFbBlocksPerSm = 3;  // resident CTAs per SM (registers)
 constexpr int kFbChunk = 2048;
 constexpr int kFbBuf = 2 * kFbChunk;  // buffered keys beyond k
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kFbThreads)
+__global__ void __launch_bounds__(kFbThreads, kFbBlocksPerSm)
 prefill_overflow_rows(PrefillArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int k = a.k;
   const int lane = threadIdx.x & 31;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);      // [k + kFbBuf]
-  float* q = reinterpret_cast<float*>(keys + k + kFbBuf);  // [D]
+  float* q = reinterpret_cast<float*>(smem);               // [D], 16-byte aligned
+  uint64_t* keys = reinterpret_cast<uint64_t*>(q + D);     // [k + kFbBuf]
   __shared__ int s_n, s_kk, s_w;
   __shared__ uint64_t s_T;
   __shared__ SelectState<1> st;
@@ -114,16 +133,27 @@ prefill_overflow_rows(PrefillArgs a) {
         const int j = c0 + jj0 + (int)threadIdx.x;
         uint64_t key = 0ull;
         if (j <= hi) {
-          // the key row in 16-byte pieces, all loads issued before the FMAs
+          // the key row in 16-byte pieces, every load issued before the
+          // first FMA (the compiler otherwise keeps a few in flight: the
+          // loop then waits on memory once per piece); q as 16-byte reads
           RawRow<T, D> kr;
           kr.load(Kg + (size_t)j * D);
-          float kf[D];
-          kr.to_f32(kf);
+          asm volatile("" ::: "memory");
+          const float4* q4 = reinterpret_cast<const float4*>(q);
           float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int e = 0; e < D; e += 2) {
-            a0 = fmaf(q[e], kf[e], a0);
-            a1 = fmaf(q[e + 1], kf[e + 1], a1);
+          for (int c = 0; c < RawRow<T, D>::kWords; ++c) {
+            constexpr int EPW = 16 / (int)sizeof(T);  // elements per piece
+            float f[EPW];
+            kr.piece_f32(c, f);
+#pragma unroll
+            for (int e = 0; e < EPW; e += 4) {
+              const float4 qv = q4[(c * EPW + e) / 4];
+              a0 = fmaf(qv.x, f[e], a0);
+              a1 = fmaf(qv.y, f[e + 1], a1);
+              a0 = fmaf(qv.z, f[e + 2], a0);
+              a1 = fmaf(qv.w, f[e + 3], a1);
+            }
           }
           key = make_key(a0 + a1, (uint32_t)j);
         }
@@ -974,12 +1004,13 @@ bool want_mass(const PrefillArgs& a) {
 template <int D>
 cudaError_t launch_overflow_d(const PrefillArgs& a, cudaStream_t s) {
   const size_t fb_smem = (size_t)(a.k + kFbBuf) * 8 + D * 4;
-  // A listed row is one CTA's job, latency-bound on its key-row loads: four
-  // CTAs per SM keep more rows in flight (the row count is only known on the
+  // A listed row is one CTA's job, latency-bound on its key-row loads: 512
+  // threads per row and every resident CTA slot of the GPU (three per SM)
+  // keep the most loads in flight (the row count is only known on the
   // device; CTAs without a row leave at once).
   prof_before(s, "prefill_overflow_rows");
   prefill_overflow_rows<__nv_bfloat16, D>
-      <<<4 * sm_count(), kFbThreads, fb_smem, s>>>(a);
+      <<<kFbBlocksPerSm * sm_count(), kFbThreads, fb_smem, s>>>(a);
   prof_after(s);
   return cudaGetLastError();
 }
