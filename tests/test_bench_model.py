@@ -50,3 +50,14 @@ def test_prefill_gather_bytes_at_8k():
 def test_step_units_are_tokens():
     assert bench.step_units(workloads.get("decode_131k")) == 1
     assert bench.step_units(workloads.get("prefill_gpt2s_8k")) == 4 * 8192
+
+
+def test_capture_hash_follows_code_only():
+    # a recorded ncu capture stays valid across comment and layout edits and
+    # is voided by any code edit
+    code = "int f(int x) {\n  return x + 1;  // one more\n}\n"
+    same = "/* header */\nint f(int x) {\n    return x + 1;\n}  // end\n"
+    other = "int f(int x) {\n  return x + 2;  // one more\n}\n"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
+    assert bench._code_only('asm("mov.u32 %0, %1;")') == 'asm("mov.u32 %0, %1;")'
