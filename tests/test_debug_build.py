@@ -119,3 +119,18 @@ def test_debug_build_full_size_matches_release(dlib, name):
         binding.use_library(prev)
     for a, b in zip(rel, dbg):
         assert np.array_equal(a, b)
+
+
+def test_debug_library_selected_by_environment(dlib):
+    # a fresh interpreter with CONDENSATE_ATTN_DEBUG=1 loads the debug build
+    import os
+    import subprocess
+    import sys
+    code = ("import sparse_transformer_attention_b200.binding as b; "
+            "print(b.LIB_PATH == b.DEBUG_LIB_PATH, "
+            "b.load().condensate_attn_build_flags())")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CONDENSATE_ATTN_DEBUG="1", PYTHONPATH=root)
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=root,
+                         capture_output=True, text=True, timeout=300)
+    assert out.stdout.split() == ["True", "1"], out.stderr[-2000:]
